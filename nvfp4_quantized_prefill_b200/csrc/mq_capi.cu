@@ -1,0 +1,422 @@
+// mq_capi.cu -- the C ABI of libmq (declared in include/mq.h): argument
+// checks, the dual-precision weight handle, workspace carving and launches.
+//
+// The phase-aware scheme (Mix-Quant, zingnex.cn forum post, section
+// "动态精度切换"; gist.science technical summary, section 2): weights are
+// stored once in a form that serves both phases -- here a handle holding the
+// BF16 matrix for decode and its NVFP4 copy for prefill -- and activations are
+// converted (quantized) at the phase boundary on every prefill call.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "mq.h"
+#include "mq_internal.h"
+
+// Per-device word in which kernels latch asynchronous errors (bounded waits
+// that ran out).  Read and cleared by mq_check.
+__device__ unsigned int g_mq_device_error;
+
+struct mq_weight {
+    int device;
+    int64_t N, K;
+    void *base;          // the one device allocation below
+    void *bf16;          // [N, K] BF16
+    uint8_t *codes;      // [N, K/2]
+    uint8_t *sf;         // swizzled scales, mq_sf_bytes(N, K)
+    float *s_enc;        // device scalar
+    float *partials;     // MQ_AMAX_PARTIALS_MAX floats (pack-time scratch)
+    CUtensorMap tmap;    // TMA map over the codes
+};
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool init = false;
+    bool supported = false;
+    int num_sms = 0;
+    unsigned *err = nullptr;
+};
+
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+size_t align256(size_t v) { return (v + 255) / 256 * 256; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+mq_status device_info(DeviceInfo **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    DeviceInfo &d = g_dev[dev];
+    if (!d.init) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return MQ_ERR_CUDA;
+        d.supported = (major == 10 && minor == 0);
+        if (d.supported) {
+            void *p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_mq_device_error) != cudaSuccess) return MQ_ERR_CUDA;
+            d.err = static_cast<unsigned *>(p);
+        }
+        d.init = true;
+    }
+    if (!d.supported) return MQ_ERR_UNSUPPORTED_DEVICE;
+    *out = &d;
+    return MQ_OK;
+}
+
+mq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MQ_OK : MQ_ERR_CUDA; }
+
+// Workspace carve for one [M, K] activation: codes | scales | partials | s_enc.
+struct ActWs {
+    uint8_t *codes;
+    uint8_t *sf;
+    float *partials;
+    float *s_enc;
+    size_t bytes;
+};
+
+size_t act_ws_bytes(int64_t M, int64_t K) {
+    return align256(static_cast<size_t>(M) * static_cast<size_t>(K / 2)) +
+           align256(mq_sf_bytes(M, K)) + align256(sizeof(float) * MQ_AMAX_PARTIALS_MAX) + 256;
+}
+
+ActWs carve_act(uint8_t *base, int64_t M, int64_t K) {
+    ActWs w;
+    size_t off = 0;
+    w.codes = base + off;
+    off += align256(static_cast<size_t>(M) * static_cast<size_t>(K / 2));
+    w.sf = base + off;
+    off += align256(mq_sf_bytes(M, K));
+    w.partials = reinterpret_cast<float *>(base + off);
+    off += align256(sizeof(float) * MQ_AMAX_PARTIALS_MAX);
+    w.s_enc = reinterpret_cast<float *>(base + off);
+    off += 256;
+    w.bytes = off;
+    return w;
+}
+
+// Shapes the kernels index with 32-bit arithmetic.
+bool shape_fits(int64_t M, int64_t K) {
+    return M >= 1 && K >= 64 && M <= (1LL << 30) && K <= (1LL << 24) &&
+           M * (K / 8) < (1LL << 32) - 1;
+}
+
+mq_status quantize_impl(DeviceInfo *d, const void *x, int64_t M, int64_t K, int64_t ldx,
+                        uint8_t *codes, uint8_t *sf, float *s_enc, const float *partials,
+                        int n_partials, float *scratch_partials, cudaStream_t s) {
+    if (!partials) {
+        const int g = mq::amax_grid(M, K, d->num_sms);
+        cudaError_t e = mq::launch_amax(x, M, K, ldx, scratch_partials, g, s);
+        if (e != cudaSuccess) return MQ_ERR_CUDA;
+        partials = scratch_partials;
+        n_partials = g;
+    }
+    return cuda_status(
+        mq::launch_quantize(x, M, K, ldx, partials, n_partials, codes, sf, s_enc, d->num_sms, s));
+}
+
+mq_status gemm_impl(DeviceInfo *d, const uint8_t *a_codes, const uint8_t *a_sf,
+                    const float *a_s_enc, int64_t M, const mq_weight *w, void *y, int64_t ldy,
+                    bool swiglu, float *amax_partials, int *n_partials, cudaStream_t s) {
+    CUtensorMap ta;
+    if (!mq::encode_codes_tmap(&ta, a_codes, M, w->K)) return MQ_ERR_CUDA;
+    mq::GemmArgs a;
+    a.sfa = a_sf;
+    a.sfb = w->sf;
+    a.s_enc_a = a_s_enc;
+    a.s_enc_b = w->s_enc;
+    a.y = y;
+    a.ldy = ldy;
+    a.M = static_cast<int>(M);
+    a.N = static_cast<int>(w->N);
+    a.K = static_cast<int>(w->K);
+    a.amax_partials = amax_partials;
+    a.err = d->err;
+    int grid = 0;
+    cudaError_t e = mq::launch_gemm_nvf4(ta, w->tmap, a, swiglu, d->num_sms, &grid, s);
+    if (n_partials) *n_partials = grid;
+    return cuda_status(e);
+}
+
+mq_status check_weight(const mq_weight *w) {
+    if (!w) return MQ_ERR_INVALID_ARG;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MQ_ERR_CUDA;
+    if (dev != w->device) return MQ_ERR_INVALID_ARG;
+    return MQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *mq_status_string(mq_status s) {
+    switch (s) {
+        case MQ_OK: return "MQ_OK";
+        case MQ_ERR_INVALID_ARG: return "MQ_ERR_INVALID_ARG";
+        case MQ_ERR_SHAPE: return "MQ_ERR_SHAPE";
+        case MQ_ERR_ALIGNMENT: return "MQ_ERR_ALIGNMENT";
+        case MQ_ERR_UNSUPPORTED_DEVICE: return "MQ_ERR_UNSUPPORTED_DEVICE";
+        case MQ_ERR_OOM: return "MQ_ERR_OOM";
+        case MQ_ERR_CUDA: return "MQ_ERR_CUDA";
+        case MQ_ERR_TIMEOUT: return "MQ_ERR_TIMEOUT";
+    }
+    return "MQ_ERR_UNKNOWN";
+}
+
+mq_status mq_check(cudaStream_t stream) {
+    DeviceInfo *d = nullptr;
+    mq_status st = device_info(&d);
+    if (st != MQ_OK) return st;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return MQ_ERR_CUDA;
+    unsigned v = 0;
+    if (cudaMemcpy(&v, d->err, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return MQ_ERR_CUDA;
+    if (v != 0) {
+        const unsigned zero = 0;
+        if (cudaMemcpy(d->err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+            return MQ_ERR_CUDA;
+        return MQ_ERR_TIMEOUT;
+    }
+    return cudaGetLastError() == cudaSuccess ? MQ_OK : MQ_ERR_CUDA;
+}
+
+size_t mq_sf_bytes(int64_t rows, int64_t K) {
+    if (rows < 1 || K < 16) return 0;
+    const int64_t rp = (rows + 127) / 128 * 128;
+    const int64_t cp = ((K / 16) + 3) / 4 * 4;
+    return static_cast<size_t>(rp * cp);
+}
+
+size_t mq_workspace_bytes(int64_t M, int64_t K) {
+    if (M < 1 || K < 64) return 0;
+    return act_ws_bytes(M, K);
+}
+
+size_t mq_mlp_workspace_bytes(int64_t M, int64_t K, int64_t I) {
+    if (M < 1 || K < 64 || I < 64) return 0;
+    return act_ws_bytes(M, K) + align256(static_cast<size_t>(M) * static_cast<size_t>(I) * 2) +
+           act_ws_bytes(M, I);
+}
+
+mq_status mq_weight_pack(const void *w_bf16, int64_t N, int64_t K, cudaStream_t stream,
+                         mq_weight **out) {
+    if (!w_bf16 || !out) return MQ_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (N < 1 || K < 64 || K % 64 != 0 || !shape_fits(N, K)) return MQ_ERR_SHAPE;
+    if (!aligned16(w_bf16)) return MQ_ERR_ALIGNMENT;
+    DeviceInfo *d = nullptr;
+    mq_status st = device_info(&d);
+    if (st != MQ_OK) return st;
+    mq_weight *w = new mq_weight();
+    cudaGetDevice(&w->device);
+    w->N = N;
+    w->K = K;
+    const size_t b_bf16 = align256(static_cast<size_t>(N) * K * 2);
+    const size_t b_codes = align256(static_cast<size_t>(N) * (K / 2));
+    const size_t b_sf = align256(mq_sf_bytes(N, K));
+    const size_t b_part = align256(sizeof(float) * MQ_AMAX_PARTIALS_MAX);
+    const size_t total = b_bf16 + b_codes + b_sf + b_part + 256;
+    if (cudaMalloc(&w->base, total) != cudaSuccess) {
+        cudaGetLastError();
+        delete w;
+        return MQ_ERR_OOM;
+    }
+    uint8_t *p = static_cast<uint8_t *>(w->base);
+    w->bf16 = p;
+    w->codes = p + b_bf16;
+    w->sf = w->codes + b_codes;
+    w->partials = reinterpret_cast<float *>(w->sf + b_sf);
+    w->s_enc = reinterpret_cast<float *>(w->sf + b_sf + b_part);
+    st = MQ_OK;
+    if (cudaMemcpyAsync(w->bf16, w_bf16, static_cast<size_t>(N) * K * 2, cudaMemcpyDeviceToDevice,
+                        stream) != cudaSuccess)
+        st = MQ_ERR_CUDA;
+    if (st == MQ_OK)
+        st = quantize_impl(d, w->bf16, N, K, K, w->codes, w->sf, w->s_enc, nullptr, 0, w->partials,
+                           stream);
+    if (st == MQ_OK && !mq::encode_codes_tmap(&w->tmap, w->codes, N, K)) st = MQ_ERR_CUDA;
+    if (st != MQ_OK) {
+        cudaFree(w->base);
+        delete w;
+        return st;
+    }
+    *out = w;
+    return MQ_OK;
+}
+
+mq_status mq_weight_free(mq_weight *w) {
+    if (!w) return MQ_OK;
+    cudaError_t e = cudaFree(w->base);
+    delete w;
+    return cuda_status(e);
+}
+
+mq_status mq_weight_views(const mq_weight *w, int64_t *N, int64_t *K, const void **bf16,
+                          const uint8_t **codes, const uint8_t **sf_swizzled,
+                          const float **s_enc_dev) {
+    if (!w) return MQ_ERR_INVALID_ARG;
+    if (N) *N = w->N;
+    if (K) *K = w->K;
+    if (bf16) *bf16 = w->bf16;
+    if (codes) *codes = w->codes;
+    if (sf_swizzled) *sf_swizzled = w->sf;
+    if (s_enc_dev) *s_enc_dev = w->s_enc;
+    return MQ_OK;
+}
+
+mq_status mq_tensor_amax(const void *x_bf16, int64_t M, int64_t K, int64_t ldx,
+                         float *amax_partials, int *n_partials, cudaStream_t stream) {
+    if (!x_bf16 || !amax_partials || !n_partials) return MQ_ERR_INVALID_ARG;
+    if (M < 1 || K < 8 || K % 8 != 0 || ldx < K || !shape_fits(M, K < 64 ? 64 : K))
+        return MQ_ERR_SHAPE;
+    if (ldx % 8 != 0 || !aligned16(x_bf16) || !aligned16(amax_partials)) return MQ_ERR_ALIGNMENT;
+    DeviceInfo *d = nullptr;
+    mq_status st = device_info(&d);
+    if (st != MQ_OK) return st;
+    const int g = mq::amax_grid(M, K, d->num_sms);
+    *n_partials = g;
+    return cuda_status(mq::launch_amax(x_bf16, M, K, ldx, amax_partials, g, stream));
+}
+
+mq_status mq_quantize_nvfp4(const void *x_bf16, int64_t M, int64_t K, int64_t ldx,
+                            uint8_t *codes, uint8_t *sf_swizzled, float *s_enc_dev,
+                            const float *amax_partials, int n_partials, void *workspace,
+                            size_t ws_bytes, cudaStream_t stream) {
+    if (!x_bf16 || !codes || !sf_swizzled || !s_enc_dev) return MQ_ERR_INVALID_ARG;
+    if (M < 1 || K < 64 || K % 64 != 0 || ldx < K || !shape_fits(M, K)) return MQ_ERR_SHAPE;
+    if (ldx % 8 != 0 || !aligned16(x_bf16) || !aligned16(codes) || !aligned16(sf_swizzled) ||
+        (reinterpret_cast<uintptr_t>(s_enc_dev) & 3u))
+        return MQ_ERR_ALIGNMENT;
+    if (amax_partials) {
+        if (n_partials < 1 || n_partials > MQ_AMAX_PARTIALS_MAX) return MQ_ERR_INVALID_ARG;
+    } else {
+        if (!workspace || ws_bytes < sizeof(float) * MQ_AMAX_PARTIALS_MAX)
+            return MQ_ERR_INVALID_ARG;
+        if (!aligned16(workspace)) return MQ_ERR_ALIGNMENT;
+    }
+    DeviceInfo *d = nullptr;
+    mq_status st = device_info(&d);
+    if (st != MQ_OK) return st;
+    return quantize_impl(d, x_bf16, M, K, ldx, codes, sf_swizzled, s_enc_dev, amax_partials,
+                         n_partials, static_cast<float *>(workspace), stream);
+}
+
+mq_status mq_gemm_nvfp4(const uint8_t *a_codes, const uint8_t *a_sf_swizzled,
+                        const float *a_s_enc_dev, int64_t M, const mq_weight *w, void *y_bf16,
+                        int64_t ldy, cudaStream_t stream) {
+    if (!a_codes || !a_sf_swizzled || !a_s_enc_dev || !y_bf16) return MQ_ERR_INVALID_ARG;
+    mq_status st = check_weight(w);
+    if (st != MQ_OK) return st;
+    if (M < 1 || ldy < w->N || !shape_fits(M, w->K) || (M + 127) / 128 * ((w->N + 255) / 256) > (1LL << 31) - 1)
+        return MQ_ERR_SHAPE;
+    if (!aligned16(a_codes) || !aligned16(a_sf_swizzled) || !aligned16(y_bf16))
+        return MQ_ERR_ALIGNMENT;
+    DeviceInfo *d = nullptr;
+    st = device_info(&d);
+    if (st != MQ_OK) return st;
+    return gemm_impl(d, a_codes, a_sf_swizzled, a_s_enc_dev, M, w, y_bf16, ldy, false, nullptr,
+                     nullptr, stream);
+}
+
+mq_status mq_gemm_nvfp4_swiglu(const uint8_t *a_codes, const uint8_t *a_sf_swizzled,
+                               const float *a_s_enc_dev, int64_t M, const mq_weight *w_gate_up,
+                               void *h_bf16, float *h_amax_partials, int *n_partials,
+                               cudaStream_t stream) {
+    if (!a_codes || !a_sf_swizzled || !a_s_enc_dev || !h_bf16 || !h_amax_partials || !n_partials)
+        return MQ_ERR_INVALID_ARG;
+    mq_status st = check_weight(w_gate_up);
+    if (st != MQ_OK) return st;
+    if (M < 1 || w_gate_up->N % 256 != 0 || !shape_fits(M, w_gate_up->K)) return MQ_ERR_SHAPE;
+    if (!aligned16(a_codes) || !aligned16(a_sf_swizzled) || !aligned16(h_bf16) ||
+        !aligned16(h_amax_partials))
+        return MQ_ERR_ALIGNMENT;
+    DeviceInfo *d = nullptr;
+    st = device_info(&d);
+    if (st != MQ_OK) return st;
+    return gemm_impl(d, a_codes, a_sf_swizzled, a_s_enc_dev, M, w_gate_up, h_bf16,
+                     w_gate_up->N / 2, true, h_amax_partials, n_partials, stream);
+}
+
+mq_status mq_prefill_linear_nvfp4(const mq_weight *w, const void *x_bf16, int64_t M,
+                                  void *y_bf16, void *workspace, size_t ws_bytes,
+                                  cudaStream_t stream) {
+    if (!x_bf16 || !y_bf16 || !workspace) return MQ_ERR_INVALID_ARG;
+    mq_status st = check_weight(w);
+    if (st != MQ_OK) return st;
+    if (M < 1 || !shape_fits(M, w->K)) return MQ_ERR_SHAPE;
+    if (ws_bytes < act_ws_bytes(M, w->K)) return MQ_ERR_INVALID_ARG;
+    if (!aligned16(x_bf16) || !aligned16(y_bf16) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return MQ_ERR_ALIGNMENT;
+    DeviceInfo *d = nullptr;
+    st = device_info(&d);
+    if (st != MQ_OK) return st;
+    ActWs a = carve_act(static_cast<uint8_t *>(workspace), M, w->K);
+    st = quantize_impl(d, x_bf16, M, w->K, w->K, a.codes, a.sf, a.s_enc, nullptr, 0, a.partials,
+                       stream);
+    if (st != MQ_OK) return st;
+    return gemm_impl(d, a.codes, a.sf, a.s_enc, M, w, y_bf16, w->N, false, nullptr, nullptr,
+                     stream);
+}
+
+mq_status mq_prefill_mlp_swiglu_nvfp4(const mq_weight *w_gate_up, const mq_weight *w_down,
+                                      const void *x_bf16, int64_t M, void *y_bf16,
+                                      void *h_bf16, void *workspace, size_t ws_bytes,
+                                      cudaStream_t stream) {
+    if (!x_bf16 || !y_bf16 || !workspace) return MQ_ERR_INVALID_ARG;
+    mq_status st = check_weight(w_gate_up);
+    if (st == MQ_OK) st = check_weight(w_down);
+    if (st != MQ_OK) return st;
+    const int64_t K = w_gate_up->K, I = w_gate_up->N / 2;
+    if (M < 1 || w_gate_up->N % 256 != 0 || w_down->K != I || !shape_fits(M, K) ||
+        !shape_fits(M, I))
+        return MQ_ERR_SHAPE;
+    if (ws_bytes < mq_mlp_workspace_bytes(M, K, I)) return MQ_ERR_INVALID_ARG;
+    if (!aligned16(x_bf16) || !aligned16(y_bf16) || (h_bf16 && !aligned16(h_bf16)) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return MQ_ERR_ALIGNMENT;
+    DeviceInfo *d = nullptr;
+    st = device_info(&d);
+    if (st != MQ_OK) return st;
+    uint8_t *base = static_cast<uint8_t *>(workspace);
+    ActWs ax = carve_act(base, M, K);
+    uint8_t *h_ws = base + ax.bytes;
+    void *h = h_bf16 ? h_bf16 : h_ws;
+    ActWs ah = carve_act(h_ws + align256(static_cast<size_t>(M) * I * 2), M, I);
+    st = quantize_impl(d, x_bf16, M, K, K, ax.codes, ax.sf, ax.s_enc, nullptr, 0, ax.partials,
+                       stream);
+    if (st != MQ_OK) return st;
+    int np = 0;
+    st = gemm_impl(d, ax.codes, ax.sf, ax.s_enc, M, w_gate_up, h, I, true, ah.partials, &np,
+                   stream);
+    if (st != MQ_OK) return st;
+    st = quantize_impl(d, h, M, I, I, ah.codes, ah.sf, ah.s_enc, ah.partials, np, nullptr, stream);
+    if (st != MQ_OK) return st;
+    return gemm_impl(d, ah.codes, ah.sf, ah.s_enc, M, w_down, y_bf16, w_down->N, false, nullptr,
+                     nullptr, stream);
+}
+
+mq_status mq_decode_linear_bf16(const mq_weight *w, const void *x_bf16, int64_t M, void *y_bf16,
+                                cudaStream_t stream) {
+    if (!x_bf16 || !y_bf16) return MQ_ERR_INVALID_ARG;
+    mq_status st = check_weight(w);
+    if (st != MQ_OK) return st;
+    if (M < 1 || M > (1LL << 20)) return MQ_ERR_SHAPE;
+    if (!aligned16(x_bf16) || !aligned16(y_bf16)) return MQ_ERR_ALIGNMENT;
+    DeviceInfo *d = nullptr;
+    st = device_info(&d);
+    if (st != MQ_OK) return st;
+    (void)d;
+    return cuda_status(mq::launch_decode(x_bf16, M, w->bf16, w->N, w->K, y_bf16, stream));
+}
+
+}  // extern "C"

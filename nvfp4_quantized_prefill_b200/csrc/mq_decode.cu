@@ -1,0 +1,109 @@
+// mq_decode.cu -- BF16 decode linear Y = X * W^T for a handful of tokens.
+//
+// Method: Mix-Quant keeps decoding in BF16 on the original weights
+// (gist.science technical summary, section 2 "Hybrid Precision Strategy");
+// the same weight handle that feeds the NVFP4 prefill GEMM keeps a BF16 copy
+// for this path, so the phase switch costs nothing.
+//
+// The op is bound by streaming W from HBM once (2 N K bytes).  Each CTA owns
+// 16 rows of W and its 8 warps split K; a warp reads, per step, 64 contiguous
+// bytes of each of its 16 rows (16-byte vector loads) plus the matching 64
+// bytes of each X row, and feeds them to two m16n8k16 BF16 MMAs (FP32
+// accumulate) with W rows as the M dimension and up to 8 X rows as N.  Both
+// fragments take the same K permutation (the 8 elements a thread loads), so no
+// shuffles or shared-memory staging are needed; for 8 tokens the tensor core
+// does the 8 FMAs per weight element that would otherwise saturate the FP32
+// pipes.  The cross-warp sum goes through shared memory.
+#include <cuda_bf16.h>
+
+#include "mq_internal.h"
+
+namespace mq {
+
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kRows = 16;
+
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32"
+        " {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__global__ void __launch_bounds__(kWarps * 32) decode_kernel(const uint4 *__restrict__ x, int M,
+                                                             const uint4 *__restrict__ w, int N,
+                                                             int K, __nv_bfloat16 *__restrict__ y) {
+    __shared__ float part[kWarps][128];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t4 = lane & 3;
+    const int n0 = blockIdx.x * kRows;
+    const int vpr = K / 8;               // 16-byte vectors per row
+    const int steps = K / 32;            // 32 K-elements per step (2 MMAs)
+    const int s0 = static_cast<int>(static_cast<int64_t>(steps) * warp / kWarps);
+    const int s1 = static_cast<int>(static_cast<int64_t>(steps) * (warp + 1) / kWarps);
+    const bool ra = n0 + g < N, rb = n0 + g + 8 < N, rx = g < M;
+    const uint4 *wa = w + static_cast<int64_t>(ra ? n0 + g : 0) * vpr + t4;
+    const uint4 *wb = w + static_cast<int64_t>(rb ? n0 + g + 8 : 0) * vpr + t4;
+    const uint4 *xr = x + static_cast<int64_t>(rx ? g : 0) * vpr + t4;
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+    int s = s0;
+    for (; s + 4 <= s1; s += 4) {
+        uint4 va[4], vb[4], vx[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            va[u] = ra ? __ldg(wa + (s + u) * 4) : z;
+            vb[u] = rb ? __ldg(wb + (s + u) * 4) : z;
+            vx[u] = rx ? __ldg(xr + (s + u) * 4) : z;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            mma_bf16_16816(c, va[u].x, vb[u].x, va[u].y, vb[u].y, vx[u].x, vx[u].y);
+            mma_bf16_16816(c, va[u].z, vb[u].z, va[u].w, vb[u].w, vx[u].z, vx[u].w);
+        }
+    }
+    for (; s < s1; ++s) {
+        const uint4 va = ra ? __ldg(wa + s * 4) : z;
+        const uint4 vb = rb ? __ldg(wb + s * 4) : z;
+        const uint4 vx = rx ? __ldg(xr + s * 4) : z;
+        mma_bf16_16816(c, va.x, vb.x, va.y, vb.y, vx.x, vx.y);
+        mma_bf16_16816(c, va.z, vb.z, va.w, vb.w, vx.z, vx.w);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) part[warp][lane * 4 + i] = c[i];
+    __syncthreads();
+    if (threadIdx.x < 128) {
+        const int q = threadIdx.x;
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < kWarps; ++i) acc += part[i][q];
+        // accumulator element q = 4 * lane' + i': row g' (+8 for i' >= 2), col 2 t4' + (i' & 1)
+        const int lq = q >> 2, iq = q & 3;
+        const int wrow = n0 + (lq >> 2) + ((iq >> 1) << 3);
+        const int m = 2 * (lq & 3) + (iq & 1);
+        if (m < M && wrow < N) y[static_cast<int64_t>(m) * N + wrow] = __float2bfloat16_rn(acc);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const void *x, int64_t M, const void *w, int64_t N, int64_t K, void *y,
+                          cudaStream_t s) {
+    const int grid = static_cast<int>((N + kRows - 1) / kRows);
+    for (int64_t m0 = 0; m0 < M; m0 += 8) {
+        const int mg = static_cast<int>(M - m0 < 8 ? M - m0 : 8);
+        decode_kernel<<<grid, kWarps * 32, 0, s>>>(
+            static_cast<const uint4 *>(x) + m0 * (K / 8), mg, static_cast<const uint4 *>(w),
+            static_cast<int>(N), static_cast<int>(K),
+            static_cast<__nv_bfloat16 *>(y) + m0 * N);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace mq

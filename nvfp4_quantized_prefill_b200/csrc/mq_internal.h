@@ -1,0 +1,54 @@
+// mq_internal.h -- launchers shared between the kernel translation units and
+// the C-ABI layer.  Not part of the public interface.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace mq {
+
+// ---- activation / weight quantization (mq_quant.cu) ------------------------
+
+// Number of CTAs (= partial maxima) the amax kernel uses for an [M, K] input.
+int amax_grid(int64_t M, int64_t K, int num_sms);
+
+// Writes `grid` partial maxima of |x| (x: BF16 [M, K], leading dimension ldx).
+cudaError_t launch_amax(const void *x, int64_t M, int64_t K, int64_t ldx, float *partials,
+                        int grid, cudaStream_t s);
+
+// NVFP4 quantization with the tensor amax = max(partials[0..n_partials)).
+cudaError_t launch_quantize(const void *x, int64_t M, int64_t K, int64_t ldx,
+                            const float *partials, int n_partials, uint8_t *codes,
+                            uint8_t *sf_swizzled, float *s_enc, int num_sms, cudaStream_t s);
+
+// ---- block-scaled GEMM (mq_gemm.cu) ------------------------------------------
+
+struct GemmArgs {
+    const uint8_t *sfa;       // swizzled scales of A (activation)
+    const uint8_t *sfb;       // swizzled scales of B (weight)
+    const float *s_enc_a;     // device scalars
+    const float *s_enc_b;
+    void *y;                  // BF16 output
+    int64_t ldy;              // output leading dimension (elements)
+    int M, N, K;              // N = weight rows (gate+up rows with SwiGLU)
+    float *amax_partials;     // SwiGLU: one max |h| per CTA
+    unsigned *err;            // device error word
+};
+
+// Launches the tcgen05 GEMM; *grid_out receives the CTA count (the number of
+// amax partials written in SwiGLU mode).
+cudaError_t launch_gemm_nvf4(const CUtensorMap &tmap_a, const CUtensorMap &tmap_b,
+                             const GemmArgs &a, bool swiglu, int num_sms, int *grid_out,
+                             cudaStream_t s);
+
+// Host-side tensor map over an [rows, K/2]-byte code matrix, 128 x 128-byte
+// boxes with 128-byte swizzle.
+bool encode_codes_tmap(CUtensorMap *map, const void *codes, int64_t rows, int64_t K);
+
+// ---- BF16 decode (mq_decode.cu) ------------------------------------------------
+
+cudaError_t launch_decode(const void *x, int64_t M, const void *w, int64_t N, int64_t K,
+                          void *y, cudaStream_t s);
+
+}  // namespace mq

@@ -1,0 +1,82 @@
+"""Host-side checks of the C ABI: libmq.so builds, loads and exports every
+symbol declared in include/mq.h; the binding declares the same set; argument
+errors are reported before any device work.  No kernel runs here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from nvfp4_quantized_prefill_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "mq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return set(re.findall(r"\b(mq_[a-z0-9_]+)\s*\(", src))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.lib()
+
+
+def test_header_declares_expected_entry_points():
+    names = header_functions()
+    for n in ["mq_quantize_nvfp4", "mq_prefill_linear_nvfp4", "mq_decode_linear_bf16",
+              "mq_weight_pack", "mq_weight_free", "mq_gemm_nvfp4", "mq_check"]:
+        assert n in names
+
+
+def test_library_exports_every_header_symbol(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_binding_covers_header(lib):
+    assert {n for n, _, _ in binding.SIGNATURES} == header_functions()
+
+
+def test_status_strings(lib):
+    for code, name in binding.STATUS.items():
+        assert binding.mq_status_string(code) == name
+
+
+def test_size_queries(lib):
+    # rows padded to 128, K/16 scales padded to a multiple of 4
+    assert binding.mq_sf_bytes(128, 256) == 128 * 16
+    assert binding.mq_sf_bytes(1, 64) == 128 * 4
+    assert binding.mq_sf_bytes(200, 320) == 256 * 20
+    assert binding.mq_sf_bytes(0, 64) == 0
+    ws = binding.mq_workspace_bytes(8192, 4096)
+    assert ws >= 8192 * 2048 + 8192 * 256 + 4 * binding.MQ_AMAX_PARTIALS_MAX
+    assert binding.mq_workspace_bytes(0, 4096) == 0
+    assert binding.mq_mlp_workspace_bytes(128, 256, 512) >= (
+        binding.mq_workspace_bytes(128, 256) + 128 * 512 * 2 + binding.mq_workspace_bytes(128, 512))
+
+
+def test_argument_errors_before_device_work(lib):
+    L = lib
+    # null pointers
+    assert L.mq_prefill_linear_nvfp4(None, None, 8, None, None, 0, None) == 1
+    assert L.mq_decode_linear_bf16(None, None, 1, None, None) == 1
+    assert L.mq_gemm_nvfp4(None, None, None, 8, None, None, 8, None) == 1
+    h = ctypes.c_void_p()
+    assert L.mq_weight_pack(None, 64, 64, None, ctypes.byref(h)) == 1
+    # shape errors: K not a multiple of 64, N < 1
+    assert L.mq_weight_pack(16, 64, 100, None, ctypes.byref(h)) == 2
+    assert L.mq_weight_pack(16, 0, 64, None, ctypes.byref(h)) == 2
+    # misaligned weight pointer
+    assert L.mq_weight_pack(17, 64, 64, None, ctypes.byref(h)) == 3
+    n = ctypes.c_int()
+    assert L.mq_tensor_amax(16, 0, 64, 64, 16, ctypes.byref(n), None) == 2
+    assert L.mq_tensor_amax(24, 4, 64, 64, 16, ctypes.byref(n), None) == 3
+    assert L.mq_quantize_nvfp4(16, 4, 96, 96, 16, 16, 16, None, 0, 16, 1 << 20, None) == 2
+    assert L.mq_quantize_nvfp4(16, 4, 64, 64, 16, 16, 16, None, 0, None, 0, None) == 1
+    assert L.mq_quantize_nvfp4(16, 4, 64, 64, 16, 16, 16, 16, 0, None, 0, None) == 1
+    assert L.mq_weight_free(None) == 0
+    assert L.mq_weight_views(None, None, None, None, None, None, None) == 1
