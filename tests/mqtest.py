@@ -76,11 +76,11 @@ def sample_rows(M: int, n: int, seed: int):
 
 
 class _DevBuf:
-    """__cuda_array_interface__ view of a raw device pointer (read-only use)."""
+    """__cuda_array_interface__ view of a raw device pointer (the caller only reads it)."""
 
     def __init__(self, ptr: int, nbytes: int):
         self.__cuda_array_interface__ = {"shape": (nbytes,), "typestr": "|u1",
-                                         "data": (ptr, True), "version": 3}
+                                         "data": (ptr, False), "version": 3}
 
 
 def fetch_device(ptr: int, nbytes: int) -> np.ndarray:
