@@ -175,6 +175,35 @@ mq_status mq_prefill_mlp_swiglu_nvfp4(const mq_weight *w_gate_up, const mq_weigh
                                       void *h_bf16, void *workspace, size_t ws_bytes,
                                       cudaStream_t stream);
 
+/* Size of the fixed device scratch used by mq_prefill_linear_nvfp4_noalloc. */
+#define MQ_NOALLOC_SCRATCH_BYTES ((size_t)48 << 20)
+
+/* The prefill linear layer without any device allocation, for callers that
+ * cannot allocate device memory at all: a plugin or host program that is
+ * handed only its input and output buffers and owns no allocator, or code on
+ * a latency-critical path where the implicit device synchronization of
+ * cudaMalloc / cudaFree is not acceptable.  The method's pages have no
+ * counterpart to this call; it is a deployment convenience.
+ *
+ * Same computation and arguments as mq_prefill_linear_nvfp4 minus the
+ * workspace: the quantized activation (codes, scales, amax partials, tensor
+ * scale) lives in one fixed array of MQ_NOALLOC_SCRATCH_BYTES (48 MiB) in the
+ * library's device memory, which every GPU that loads libmq keeps until the
+ * process exits.  Requests whose workspace would exceed it --
+ * mq_workspace_bytes(M, K) > MQ_NOALLOC_SCRATCH_BYTES, e.g. more than about
+ * 21800 tokens at K = 4096 -- return MQ_ERR_SHAPE before any work is queued.
+ * Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current); make that first call before any stream capture begins.
+ * All calls on a device share the one array and it keeps the last call's
+ * contents (every byte a call reads is written earlier in the same call, so
+ * nothing needs clearing).  Calls whose work overlaps on the GPU -- on two
+ * streams without ordering, or from two host threads -- race on the array and
+ * corrupt each other's results; serialize them. */
+mq_status mq_prefill_linear_nvfp4_noalloc(const mq_weight *w, const void *x_bf16, int64_t M,
+                                          void *y_bf16, cudaStream_t stream);
+
 /* ---- decode (gist.science §2: decoding keeps BF16) ----------------------- */
 
 /* BF16 decode linear on the handle's BF16 copy: y[m, n] = bf16( sum_k x[m,k]

@@ -36,6 +36,7 @@ SIGNATURES = [
     ("mq_prefill_linear_nvfp4", _I, [_P, _P, _I64, _P, _P, _SZ, _P]),
     ("mq_mlp_workspace_bytes", _SZ, [_I64, _I64, _I64]),
     ("mq_prefill_mlp_swiglu_nvfp4", _I, [_P, _P, _P, _I64, _P, _P, _P, _SZ, _P]),
+    ("mq_prefill_linear_nvfp4_noalloc", _I, [_P, _P, _I64, _P, _P]),
     ("mq_decode_linear_bf16", _I, [_P, _P, _I64, _P, _P]),
 ]
 
@@ -164,6 +165,11 @@ def mq_prefill_mlp_swiglu_nvfp4(w_gate_up: int, w_down: int, x, M: int, y, h, wo
     _ok("mq_prefill_mlp_swiglu_nvfp4", lib().mq_prefill_mlp_swiglu_nvfp4(
         w_gate_up, w_down, _ptr(x), M, _ptr(y), _ptr(h), _ptr(workspace), ws_bytes,
         _stream(stream)))
+
+
+def mq_prefill_linear_nvfp4_noalloc(weight: int, x, M: int, y, stream=None) -> None:
+    _ok("mq_prefill_linear_nvfp4_noalloc", lib().mq_prefill_linear_nvfp4_noalloc(
+        weight, _ptr(x), M, _ptr(y), _stream(stream)))
 
 
 def mq_decode_linear_bf16(weight: int, x, M: int, y, stream=None) -> None:

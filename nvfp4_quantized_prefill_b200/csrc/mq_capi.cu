@@ -405,6 +405,60 @@ mq_status mq_prefill_mlp_swiglu_nvfp4(const mq_weight *w_gate_up, const mq_weigh
                      nullptr, stream);
 }
 
+}  // extern "C"
+
+// ---- fixed scratch for the allocation-free prefill entry point -------------
+// One array per device, part of this library's device image: the driver
+// places it when the library's device code is loaded, so a caller never
+// allocates it.  Host code cannot use the symbol as a pointer; its device
+// address is looked up once per device below.
+static __device__ __align__(256) uint8_t g_mq_noalloc_scratch[MQ_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+uint8_t *g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+mq_status noalloc_scratch(uint8_t **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_mq_noalloc_scratch) != cudaSuccess || !p)
+            return MQ_ERR_CUDA;
+        g_noalloc_ptr[dev] = static_cast<uint8_t *>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return MQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+mq_status mq_prefill_linear_nvfp4_noalloc(const mq_weight *w, const void *x_bf16, int64_t M,
+                                          void *y_bf16, cudaStream_t stream) {
+    if (!x_bf16 || !y_bf16) return MQ_ERR_INVALID_ARG;
+    mq_status st = check_weight(w);
+    if (st != MQ_OK) return st;
+    if (M < 1 || !shape_fits(M, w->K)) return MQ_ERR_SHAPE;
+    if (act_ws_bytes(M, w->K) > MQ_NOALLOC_SCRATCH_BYTES) return MQ_ERR_SHAPE;
+    if (!aligned16(x_bf16) || !aligned16(y_bf16)) return MQ_ERR_ALIGNMENT;
+    DeviceInfo *d = nullptr;
+    st = device_info(&d);
+    if (st != MQ_OK) return st;
+    uint8_t *scratch = nullptr;
+    st = noalloc_scratch(&scratch);
+    if (st != MQ_OK) return st;
+    ActWs a = carve_act(scratch, M, w->K);
+    st = quantize_impl(d, x_bf16, M, w->K, w->K, a.codes, a.sf, a.s_enc, nullptr, 0, a.partials,
+                       stream);
+    if (st != MQ_OK) return st;
+    return gemm_impl(d, a.codes, a.sf, a.s_enc, M, w, y_bf16, w->N, false, nullptr, nullptr,
+                     stream);
+}
+
 mq_status mq_decode_linear_bf16(const mq_weight *w, const void *x_bf16, int64_t M, void *y_bf16,
                                 cudaStream_t stream) {
     if (!x_bf16 || !y_bf16) return MQ_ERR_INVALID_ARG;
