@@ -37,7 +37,12 @@ constexpr uint32_t kSfbBytes = 2 * 4 * 512;      // two 128-row halves
 constexpr uint32_t kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // 55296
 constexpr uint32_t kBarBytes = 256;
 constexpr uint32_t kSmemBytes = kStages * kStageBytes + kBarBytes + 1024;
-constexpr int kThreads = 320;
+#ifndef MQ_GEMM_COPIERS
+#define MQ_GEMM_COPIERS 2
+#endif
+constexpr int kCopiers = MQ_GEMM_COPIERS;        // scale-copy warps
+constexpr int kEpiWarp0 = 2 + kCopiers;          // first of 8 epilogue warps
+constexpr int kThreads = 32 * (kEpiWarp0 + 8);
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfCol = 256;                 // scale columns follow the accumulator
 constexpr uint32_t kSfColsPerStage = 48;         // 16 for A + 32 for B
@@ -135,7 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kStages + 3);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * kStages + 4);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     float *red = reinterpret_cast<float *>(tmem_slot + 2);  // 8 floats
 
@@ -145,6 +150,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t acc_full = bar0 + 8u * (2 * kStages);
     const uint32_t acc_empty = acc_full + 8u;
     const uint32_t drain_bar = acc_full + 16u;
+    const uint32_t sf_drain_bar = acc_full + 24u;
+    const uint32_t sf_full0 = acc_full + 32u;     // sf_full[s] = sf_full0 + 8 s
     const uint32_t smem0 = smem_u32(smem);
 
     if (threadIdx.x == 0) {
@@ -155,6 +162,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 8);
         mbar_init(drain_bar, 1);
+        mbar_init(sf_drain_bar, kCopiers);
+        for (int s = 0; s < kStages; ++s) mbar_init(sf_full0 + 8u * s, kCopiers);
         *abort_flag = 0;
         fence_barrier_init();
         prefetch_tmap(&tmap_a);
@@ -228,7 +237,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag, p.err)) break;
                 tc_fence_after();
                 for (int kt = 0; kt < p.k_tiles; ++kt) {
-                    if (!mbar_wait(bar0 + 8u * stage, phase, abort_flag, p.err)) {
+                    // operands landed and this stage's scales are in TMEM
+                    if (!mbar_wait(sf_full0 + 8u * stage, phase, abort_flag, p.err)) {
                         ok = false;
                         break;
                     }
@@ -236,15 +246,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int natoms = min(4, p.sf_ktiles - kt * 4);
                     const uint32_t sA = smem0 + stage * kStageBytes;
                     const uint32_t sB = sA + kABytes;
-                    const uint32_t sSFA = sB + kBBytes;
-                    const uint32_t sSFB = sSFA + kSfaBytes;
                     const uint32_t tsfa = tmem + kSfCol + stage * kSfColsPerStage;
                     const uint32_t tsfb = tsfa + 16u;
-                    for (int a = 0; a < natoms; ++a) {
-                        tc_cp_sf(tsfa + 4u * a, sdesc_sf_tile(sSFA + 512u * a));
-                        tc_cp_sf(tsfb + 8u * a, sdesc_sf_tile(sSFB + 512u * a));
-                        tc_cp_sf(tsfb + 8u * a + 4u, sdesc_sf_tile(sSFB + 4u * 512u + 512u * a));
-                    }
                     for (int kb = 0; kb < natoms; ++kb) {
                         tc_mma_nvf4(tmem, sdesc_kmajor_sw128(sA + 32u * kb),
                                     sdesc_kmajor_sw128(sB + 32u * kb), idesc, tsfa + 4u * kb,
@@ -264,9 +267,48 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_commit(drain_bar);
             drain_wait(drain_bar, 0, p.err);
         }
+    } else if (warp < kEpiWarp0) {
+        // ------------------------------------------------------------ scale copiers
+        // Each copier warp copies its share of a stage's scale tiles (k-blocks
+        // c, c + kCopiers, ...) smem -> TMEM with tcgen05.cp from its own
+        // thread: a thread's tcgen05 instructions run in order, so copies
+        // issued by the MMA thread would queue in front of its MMAs.  Each
+        // copier arrives on sf_full[stage] once its copies have landed.
+        const int cid = warp - 2;
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+                for (int kt = 0; kt < p.k_tiles; ++kt) {
+                    if (!mbar_wait(bar0 + 8u * stage, phase, abort_flag, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int natoms = min(4, p.sf_ktiles - kt * 4);
+                    const uint32_t sSFA = smem0 + stage * kStageBytes + kABytes + kBBytes;
+                    const uint32_t sSFB = sSFA + kSfaBytes;
+                    const uint32_t tsfa = tmem + kSfCol + stage * kSfColsPerStage;
+                    const uint32_t tsfb = tsfa + 16u;
+                    for (int a = cid; a < natoms; a += kCopiers) {
+                        tc_cp_sf(tsfa + 4u * a, sdesc_sf_tile(sSFA + 512u * a));
+                        tc_cp_sf(tsfb + 8u * a, sdesc_sf_tile(sSFB + 512u * a));
+                        tc_cp_sf(tsfb + 8u * a + 4u, sdesc_sf_tile(sSFB + 4u * 512u + 512u * a));
+                    }
+                    tc_commit(sf_full0 + 8u * stage);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            tc_commit(sf_drain_bar);
+            drain_wait(sf_drain_bar, 0, p.err);
+        }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int ew = warp - 2;         // 0..7
+        const int ew = warp - kEpiWarp0; // 0..7
         const int sub = warp & 3;        // TMEM lane group this warp may read
         const int half = ew >> 2;        // column half of the tile
         const float alpha = __frcp_rn(__fmul_rn(*p.s_enc_a, *p.s_enc_b));
