@@ -30,6 +30,7 @@ struct mq_weight {
     float *s_enc;        // device scalar
     float *partials;     // MQ_AMAX_PARTIALS_MAX floats (pack-time scratch)
     CUtensorMap tmap;    // TMA map over the codes
+    CUtensorMap tmap_sf; // TMA map over the swizzled scales
 };
 
 namespace {
@@ -128,11 +129,10 @@ mq_status quantize_impl(DeviceInfo *d, const void *x, int64_t M, int64_t K, int6
 mq_status gemm_impl(DeviceInfo *d, const uint8_t *a_codes, const uint8_t *a_sf,
                     const float *a_s_enc, int64_t M, const mq_weight *w, void *y, int64_t ldy,
                     bool swiglu, float *amax_partials, int *n_partials, cudaStream_t s) {
-    CUtensorMap ta;
+    CUtensorMap ta, tsa;
     if (!mq::encode_codes_tmap(&ta, a_codes, M, w->K)) return MQ_ERR_CUDA;
+    if (!mq::encode_sf_tmap(&tsa, a_sf, M, w->K)) return MQ_ERR_CUDA;
     mq::GemmArgs a;
-    a.sfa = a_sf;
-    a.sfb = w->sf;
     a.s_enc_a = a_s_enc;
     a.s_enc_b = w->s_enc;
     a.y = y;
@@ -143,7 +143,7 @@ mq_status gemm_impl(DeviceInfo *d, const uint8_t *a_codes, const uint8_t *a_sf,
     a.amax_partials = amax_partials;
     a.err = d->err;
     int grid = 0;
-    cudaError_t e = mq::launch_gemm_nvf4(ta, w->tmap, a, swiglu, d->num_sms, &grid, s);
+    cudaError_t e = mq::launch_gemm_nvf4(ta, w->tmap, tsa, w->tmap_sf, a, swiglu, d->num_sms, &grid, s);
     if (n_partials) *n_partials = grid;
     return cuda_status(e);
 }
@@ -244,7 +244,9 @@ mq_status mq_weight_pack(const void *w_bf16, int64_t N, int64_t K, cudaStream_t 
     if (st == MQ_OK)
         st = quantize_impl(d, w->bf16, N, K, K, w->codes, w->sf, w->s_enc, nullptr, 0, w->partials,
                            stream);
-    if (st == MQ_OK && !mq::encode_codes_tmap(&w->tmap, w->codes, N, K)) st = MQ_ERR_CUDA;
+    if (st == MQ_OK && (!mq::encode_codes_tmap(&w->tmap, w->codes, N, K) ||
+                        !mq::encode_sf_tmap(&w->tmap_sf, w->sf, N, K)))
+        st = MQ_ERR_CUDA;
     if (st != MQ_OK) {
         cudaFree(w->base);
         delete w;

@@ -7,20 +7,28 @@
 // Deployment"); decoding keeps BF16.  Y = bf16(acc / (s_enc_a * s_enc_b)),
 // acc = sum_k e2m1(a) dec(sa) e2m1(b) dec(sb), one E4M3 scale per 16 K.
 //
-// Kernel shape (one persistent CTA per SM, 10 warps):
-//   warp 0     TMA producer: A tile [128 x 256 fp4], B tile [256 x 256 fp4]
-//              (two 128-row boxes, 128-byte swizzle) and the matching 512-byte
-//              scale-factor tiles (plain bulk copies) into a 4-stage ring.
-//   warp 1     MMA issuer: copies the scale tiles into TMEM (tcgen05.cp) and
-//              issues tcgen05.mma kind::mxf4nvf4 block16, M=128 N=256 K=64,
-//              into one 128 x 256 FP32 accumulator in TMEM.
-//   warps 2-9  epilogue: drain the accumulator (tcgen05.ld), release it to
-//              the MMA warp, then scale, round to BF16 and store -- the stores
-//              overlap the next tile's main loop.
+// Kernel shape: CTA pairs (clusters of 2, one CTA per SM, persistent), each
+// pair computing 256 x 256 output tiles with the paired MMA
+// (tcgen05.mma.cta_group::2, M = 256 split 128 rows per CTA, N = 256):
+//   warp 0       (both CTAs) TMA producer: this CTA's 128 A rows and 128 B
+//                rows of a 256-wide K step (128-byte swizzle), its A scale
+//                tiles and both B scale halves, into a 5-stage ring; every
+//                load completes on the even CTA's stage barrier.
+//   warp 1       (even CTA) MMA issuer: 4 paired MMAs (K = 64 each) per stage
+//                into a 128 x 256 FP32 accumulator in each CTA's TMEM.
+//   warps 2-3    (even CTA) scale copiers: tcgen05.cp of the stage's scale
+//                tiles into both CTAs' TMEM, from their own threads -- a
+//                thread's tcgen05 instructions run in order, so copies issued
+//                by the MMA thread would queue ahead of its MMAs.
+//   warps 4-11   (both CTAs) epilogue: drain the CTA's accumulator half with
+//                tcgen05.ld, release it to the MMA thread, then scale, round to
+//                BF16 and store while the next tile's main loop runs.
 // Every mbarrier wait is bounded (about two seconds); on a timeout the kernel
-// latches an error bit, stops issuing work, lets in-flight copies and MMAs
-// land, frees its tensor memory and exits.
+// latches an error bit, stops issuing work, lets issued copies and MMAs land,
+// frees its tensor memory and exits.
 #include <cuda_bf16.h>
+
+#include <cstring>
 
 #include "mq_internal.h"
 #include "mq_ptx.cuh"
@@ -29,39 +37,50 @@ namespace mq {
 
 namespace {
 
-constexpr int kStages = 4;
-constexpr uint32_t kABytes = 128 * 128;          // 128 rows x 128 B (256 fp4)
-constexpr uint32_t kBBytes = 256 * 128;          // 256 rows x 128 B
-constexpr uint32_t kSfaBytes = 4 * 512;          // 4 scale tiles (K = 256)
-constexpr uint32_t kSfbBytes = 2 * 4 * 512;      // two 128-row halves
-constexpr uint32_t kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // 55296
-constexpr uint32_t kBarBytes = 256;
-constexpr uint32_t kSmemBytes = kStages * kStageBytes + kBarBytes + 1024;
+#ifndef MQ_GEMM_STAGES
+#define MQ_GEMM_STAGES 5
+#endif
+#ifndef MQ_GEMM_GROUP_M
+#define MQ_GEMM_GROUP_M 8
+#endif
 #ifndef MQ_GEMM_COPIERS
 #define MQ_GEMM_COPIERS 2
 #endif
-constexpr int kCopiers = MQ_GEMM_COPIERS;        // scale-copy warps
+
+constexpr int kStages = MQ_GEMM_STAGES;
+constexpr uint32_t kABytes = 128 * 128;          // this CTA's 128 A rows x 128 B (256 fp4)
+constexpr uint32_t kBBytes = 128 * 128;          // this CTA's 128 B rows
+constexpr uint32_t kSfaBytes = 4 * 512;          // 4 scale tiles (K = 256) of the A rows
+constexpr uint32_t kSfbBytes = 2 * 4 * 512;      // both 128-row halves of the B tile
+constexpr uint32_t kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // 38912
+constexpr uint32_t kPairTxBytes = 2 * kStageBytes;                           // both CTAs
+constexpr uint32_t kStageTileBytes = 32 * 128;    // epilogue staging: 32 rows x 64 bf16
+constexpr uint32_t kStagingBytes = 8 * kStageTileBytes;  // one per epilogue warp
+constexpr uint32_t kBarBytes = 256;
+constexpr uint32_t kSmemBytes = kStages * kStageBytes + kStagingBytes + kBarBytes + 1024;
+constexpr int kCopiers = MQ_GEMM_COPIERS;        // scale-copy warps (even CTA)
 constexpr int kEpiWarp0 = 2 + kCopiers;          // first of 8 epilogue warps
 constexpr int kThreads = 32 * (kEpiWarp0 + 8);
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfCol = 256;                 // scale columns follow the accumulator
 constexpr uint32_t kSfColsPerStage = 48;         // 16 for A + 32 for B
-constexpr int kGroupM = 16;                      // tile raster: 16 M-tiles per group
+constexpr int kGroupM = MQ_GEMM_GROUP_M;         // tile raster: M-tiles per group
+constexpr uint16_t kPairMask = 0x3;
 
 static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
 static_assert(kSfCol + kStages * kSfColsPerStage <= kTmemCols, "TMEM budget");
+static_assert((3 * kStages + 4) * 8 + 48 <= kBarBytes, "barrier area");
 
 struct Params {
-    const uint8_t *sfa;
-    const uint8_t *sfb;
     const float *s_enc_a;
     const float *s_enc_b;
     __nv_bfloat16 *y;
     int64_t ldy;
     int M, N, K;
-    int tiles_m, tiles_n, k_tiles, sf_ktiles, sf_rowblocks_b, n_half;
+    int tiles_m, tiles_n, k_tiles, sf_ktiles, n_half;
     float *amax_partials;
     unsigned *err;
+    int tma_store;        // 1: outputs leave through TMA stores via shared memory
 };
 
 __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int &tm, int &tn) {
@@ -72,22 +91,6 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int
     const int local = t - g * per_group;
     tm = first + local % gs;
     tn = local / gs;
-}
-
-// B rows / scale row-blocks of N-tile tn: plain mode covers weight rows
-// [256 tn, 256 tn + 256); SwiGLU mode covers gate rows [128 tn, +128) and the
-// matching up rows [n_half + 128 tn, +128).
-__device__ __forceinline__ void b_rows(const Params &p, int tn, bool swiglu, int &row0, int &row1,
-                                       int &rb0, int &rb1) {
-    if (swiglu) {
-        row0 = tn * 128;
-        row1 = p.n_half + tn * 128;
-    } else {
-        row0 = tn * 256;
-        row1 = tn * 256 + 128;
-    }
-    rb0 = row0 / 128;
-    rb1 = row1 / 128;
 }
 
 // Waits (time-bounded, ignoring the abort flag) so that in-flight asynchronous
@@ -133,48 +136,59 @@ __device__ __forceinline__ void store_row(__nv_bfloat16 *dst, const uint32_t *pa
 }
 
 template <bool kSwiglu>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                     const __grid_constant__ CUtensorMap tmap_b, const Params p) {
+                     const __grid_constant__ CUtensorMap tmap_b,
+                     const __grid_constant__ CUtensorMap tmap_sfa,
+                     const __grid_constant__ CUtensorMap tmap_sfb,
+                     const __grid_constant__ CUtensorMap tmap_y, const Params p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes + kStagingBytes);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * kStages + 4);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     float *red = reinterpret_cast<float *>(tmem_slot + 2);  // 8 floats
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const uint32_t bar0 = smem_u32(bars);
-    const uint32_t acc_full = bar0 + 8u * (2 * kStages);
+    const uint32_t rank = cluster_ctarank();         // 0: the pair's issuing CTA
+    const uint32_t bar0 = smem_u32(bars);             // full[s]  = bar0 + 8 s
+    const uint32_t empty0 = bar0 + 8u * kStages;      // empty[s]
+    const uint32_t sf_full0 = bar0 + 16u * kStages;   // sf_full[s]
+    const uint32_t acc_full = bar0 + 24u * kStages;
     const uint32_t acc_empty = acc_full + 8u;
     const uint32_t drain_bar = acc_full + 16u;
     const uint32_t sf_drain_bar = acc_full + 24u;
-    const uint32_t sf_full0 = acc_full + 32u;     // sf_full[s] = sf_full0 + 8 s
     const uint32_t smem0 = smem_u32(smem);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(bar0 + 8u * s, 1);               // full[s]
-            mbar_init(bar0 + 8u * (kStages + s), 1);   // empty[s]
+            mbar_init(bar0 + 8u * s, 1);             // arrive.expect_tx of the even CTA
+            mbar_init(empty0 + 8u * s, 1);           // MMA commit (to both CTAs)
+            mbar_init(sf_full0 + 8u * s, kCopiers);  // one commit per copier
         }
         mbar_init(acc_full, 1);
-        mbar_init(acc_empty, 8);
+        mbar_init(acc_empty, 16);                    // 8 epilogue warps x 2 CTAs
         mbar_init(drain_bar, 1);
         mbar_init(sf_drain_bar, kCopiers);
-        for (int s = 0; s < kStages; ++s) mbar_init(sf_full0 + 8u * s, kCopiers);
         *abort_flag = 0;
         fence_barrier_init();
         prefetch_tmap(&tmap_a);
         prefetch_tmap(&tmap_b);
+        prefetch_tmap(&tmap_sfa);
+        prefetch_tmap(&tmap_sfb);
+        if (p.tma_store) prefetch_tmap(&tmap_y);
     }
-    if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    if (warp == 1) tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
     tc_fence_before();
     __syncthreads();
+    cluster_sync();  // the peer's barriers exist before any cross-CTA signal
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const int num_tiles = p.tiles_m * p.tiles_n;
+    const int pair = static_cast<int>(blockIdx.x >> 1);
+    const int npairs = static_cast<int>(gridDim.x >> 1);
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -183,61 +197,66 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t phase = 0;
             uint32_t armed = 0, armed_parity = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-                int tm, tn, row0, row1, rb0, rb1;
+            for (int t = pair; t < num_tiles && ok; t += npairs) {
+                int tm, tn;
                 tile_coords(t, p.tiles_m, p.tiles_n, tm, tn);
-                b_rows(p, tn, kSwiglu, row0, row1, rb0, rb1);
-                const bool rb1_ok = rb1 < p.sf_rowblocks_b;
+                // B rows of this CTA and the two 128-row scale blocks of the tile
+                int b_row, rb0, rb1;
+                if (kSwiglu) {
+                    rb0 = tn;                            // gate rows 128 tn ..
+                    rb1 = p.n_half / 128 + tn;           // matching up rows
+                    b_row = (rank == 0 ? rb0 : rb1) * 128;
+                } else {
+                    rb0 = 2 * tn;
+                    rb1 = 2 * tn + 1;
+                    b_row = tn * 256 + static_cast<int>(rank) * 128;
+                }
+                const int a_row = tm * 256 + static_cast<int>(rank) * 128;
+                const int a_sf = (2 * tm + static_cast<int>(rank)) * p.sf_ktiles;
                 for (int kt = 0; kt < p.k_tiles; ++kt) {
-                    const uint32_t full = bar0 + 8u * stage;
-                    if (!mbar_wait(bar0 + 8u * (kStages + stage), phase ^ 1u, abort_flag, p.err)) {
+                    if (!mbar_wait(empty0 + 8u * stage, phase ^ 1u, abort_flag, p.err)) {
                         ok = false;
                         break;
                     }
-                    const int natoms = min(4, p.sf_ktiles - kt * 4);
-                    const uint32_t sf_bytes = static_cast<uint32_t>(natoms) * 512u;
-                    const uint32_t bytes =
-                        kABytes + kBBytes + sf_bytes * (rb1_ok ? 3u : 2u);
-                    mbar_arrive_expect_tx(full, bytes);
-                    armed |= 1u << stage;
-                    armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+                    const uint32_t full_local = bar0 + 8u * stage;
+                    const uint32_t full_pair = mapa_shared(full_local, 0);
+                    if (rank == 0) {
+                        mbar_arrive_expect_tx(full_local, kPairTxBytes);
+                        armed |= 1u << stage;
+                        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+                    }
                     const uint32_t sA = smem0 + stage * kStageBytes;
                     const uint32_t sB = sA + kABytes;
                     const uint32_t sSFA = sB + kBBytes;
                     const uint32_t sSFB = sSFA + kSfaBytes;
-                    tma_load_2d(sA, &tmap_a, kt * 128, tm * 128, full);
-                    tma_load_2d(sB, &tmap_b, kt * 128, row0, full);
-                    tma_load_2d(sB + 128u * 128u, &tmap_b, kt * 128, row1, full);
-                    bulk_load(sSFA, p.sfa + (static_cast<int64_t>(tm) * p.sf_ktiles + kt * 4) * 512,
-                              sf_bytes, full);
-                    bulk_load(sSFB, p.sfb + (static_cast<int64_t>(rb0) * p.sf_ktiles + kt * 4) * 512,
-                              sf_bytes, full);
-                    if (rb1_ok)
-                        bulk_load(sSFB + 4u * 512u,
-                                  p.sfb + (static_cast<int64_t>(rb1) * p.sf_ktiles + kt * 4) * 512,
-                                  sf_bytes, full);
+                    tma_load_2d_pair(sA, &tmap_a, kt * 128, a_row, full_pair);
+                    tma_load_2d_pair(sB, &tmap_b, kt * 128, b_row, full_pair);
+                    tma_load_2d_pair(sSFA, &tmap_sfa, 0, a_sf + kt * 4, full_pair);
+                    tma_load_2d_pair(sSFB, &tmap_sfb, 0, rb0 * p.sf_ktiles + kt * 4, full_pair);
+                    tma_load_2d_pair(sSFB + 4u * 512u, &tmap_sfb, 0, rb1 * p.sf_ktiles + kt * 4,
+                                     full_pair);
                     if (++stage == kStages) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
             }
-            // let every issued copy land before the CTA may exit
+            // both CTAs' loads of every armed stage land before the pair may exit
             for (int s = 0; s < kStages; ++s)
                 if (armed & (1u << s)) drain_wait(bar0 + 8u * s, (armed_parity >> s) & 1u, p.err);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc = idesc_nvf4(128, 256);
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t idesc = idesc_nvf4(256, 256);
             int stage = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+            for (int t = pair; t < num_tiles && ok; t += npairs) {
                 if (!mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag, p.err)) break;
                 tc_fence_after();
                 for (int kt = 0; kt < p.k_tiles; ++kt) {
-                    // operands landed and this stage's scales are in TMEM
+                    // operands of both CTAs landed and the stage's scales are in TMEM
                     if (!mbar_wait(sf_full0 + 8u * stage, phase, abort_flag, p.err)) {
                         ok = false;
                         break;
@@ -249,37 +268,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t tsfa = tmem + kSfCol + stage * kSfColsPerStage;
                     const uint32_t tsfb = tsfa + 16u;
                     for (int kb = 0; kb < natoms; ++kb) {
-                        tc_mma_nvf4(tmem, sdesc_kmajor_sw128(sA + 32u * kb),
-                                    sdesc_kmajor_sw128(sB + 32u * kb), idesc, tsfa + 4u * kb,
-                                    tsfb + 8u * kb, (kt | kb) != 0 ? 1u : 0u);
+                        tc_mma_nvf4_pair(tmem, sdesc_kmajor_sw128(sA + 32u * kb),
+                                         sdesc_kmajor_sw128(sB + 32u * kb), idesc, tsfa + 4u * kb,
+                                         tsfb + 8u * kb, (kt | kb) != 0 ? 1u : 0u);
                     }
-                    tc_commit(bar0 + 8u * (kStages + stage));  // frees the smem stage
+                    tc_commit_pair_mc(empty0 + 8u * stage, kPairMask);  // frees both CTAs' stage
                     if (++stage == kStages) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
                 if (!ok) break;
-                tc_commit(acc_full);
+                tc_commit_pair_mc(acc_full, kPairMask);
                 acc_phase ^= 1u;
             }
-            // every MMA / copy issued by this thread completes before TMEM is freed
-            tc_commit(drain_bar);
+            // every MMA issued by this thread completes before TMEM is freed
+            tc_commit_pair(drain_bar);
             drain_wait(drain_bar, 0, p.err);
         }
     } else if (warp < kEpiWarp0) {
         // ------------------------------------------------------------ scale copiers
-        // Each copier warp copies its share of a stage's scale tiles (k-blocks
-        // c, c + kCopiers, ...) smem -> TMEM with tcgen05.cp from its own
-        // thread: a thread's tcgen05 instructions run in order, so copies
-        // issued by the MMA thread would queue in front of its MMAs.  Each
-        // copier arrives on sf_full[stage] once its copies have landed.
+        // Copier c copies k-blocks c, c + kCopiers, ... of each stage: the A
+        // scale tile (each CTA its own rows) and both B halves, into the
+        // stage's TMEM scale slot of both CTAs, then arrives on sf_full[stage].
         const int cid = warp - 2;
-        if (lane == 0) {
+        if (lane == 0 && rank == 0) {
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+            for (int t = pair; t < num_tiles && ok; t += npairs) {
                 for (int kt = 0; kt < p.k_tiles; ++kt) {
                     if (!mbar_wait(bar0 + 8u * stage, phase, abort_flag, p.err)) {
                         ok = false;
@@ -292,36 +309,59 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t tsfa = tmem + kSfCol + stage * kSfColsPerStage;
                     const uint32_t tsfb = tsfa + 16u;
                     for (int a = cid; a < natoms; a += kCopiers) {
-                        tc_cp_sf(tsfa + 4u * a, sdesc_sf_tile(sSFA + 512u * a));
-                        tc_cp_sf(tsfb + 8u * a, sdesc_sf_tile(sSFB + 512u * a));
-                        tc_cp_sf(tsfb + 8u * a + 4u, sdesc_sf_tile(sSFB + 4u * 512u + 512u * a));
+                        tc_cp_sf_pair(tsfa + 4u * a, sdesc_sf_tile(sSFA + 512u * a));
+                        tc_cp_sf_pair(tsfb + 8u * a, sdesc_sf_tile(sSFB + 512u * a));
+                        tc_cp_sf_pair(tsfb + 8u * a + 4u, sdesc_sf_tile(sSFB + 4u * 512u + 512u * a));
                     }
-                    tc_commit(sf_full0 + 8u * stage);
+                    tc_commit_pair(sf_full0 + 8u * stage);
                     if (++stage == kStages) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
             }
-            tc_commit(sf_drain_bar);
+            tc_commit_pair(sf_drain_bar);
             drain_wait(sf_drain_bar, 0, p.err);
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int ew = warp - kEpiWarp0; // 0..7
-        const int sub = warp & 3;        // TMEM lane group this warp may read
-        const int half = ew >> 2;        // column half of the tile
+        const int ew = warp - kEpiWarp0;  // 0..7
+        const int sub = warp & 3;         // TMEM lane group this warp may read
+        const int half = ew >> 2;         // column half of the tile
         const float alpha = __frcp_rn(__fmul_rn(*p.s_enc_a, *p.s_enc_b));
         const bool vec_ok = (p.ldy % 8) == 0;
+        const uint32_t acc_empty_pair = mapa_shared(acc_empty, 0);
+        // this warp's staging tile: 32 rows of 128 bytes, 128-byte swizzled
+        // (16-byte chunk j of row r at r * 128 + ((j ^ (r % 8)) * 16)), the
+        // layout the output tensor map's SWIZZLE_128B store reads
+        const uint32_t stg = smem0 + kStages * kStageBytes + ew * kStageTileBytes;
+        const uint32_t stg_row = stg + lane * 128u;
         uint32_t acc_phase = 0;
         float hmax = 0.0f;
-        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+        // Stages 32 rows x 64 columns (this lane's row: 32 packed bf16 pairs)
+        // and stores them at output (col0, row0) with one TMA store.
+        auto tma_store_chunk = [&](const uint32_t *q, int col0, int row0) {
+            if (lane == 0) bulk_wait_group_read0();  // staging free again
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                st_shared_v4(stg_row + ((static_cast<uint32_t>(j) ^ (lane & 7u)) << 4), q[4 * j],
+                             q[4 * j + 1], q[4 * j + 2], q[4 * j + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_2d(&tmap_y, col0, row0, stg);
+                bulk_commit_group();
+            }
+        };
+        for (int t = pair; t < num_tiles; t += npairs) {
             int tm, tn;
             tile_coords(t, p.tiles_m, p.tiles_n, tm, tn);
             // warp-uniform decision: the TMEM loads below are .sync.aligned
             if (!__all_sync(0xFFFFFFFFu, mbar_wait(acc_full, acc_phase, abort_flag, p.err))) break;
             tc_fence_after();
-            const int row = tm * 128 + sub * 32 + lane;
+            const int row0 = tm * 256 + static_cast<int>(rank) * 128 + sub * 32;
+            const int row = row0 + lane;
             const uint32_t tbase = tmem + (static_cast<uint32_t>(sub * 32) << 16);
             if (!kSwiglu) {
                 uint32_t packed[64];
@@ -342,11 +382,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(acc_empty);
+                if (lane == 0) mbar_arrive_cluster(acc_empty_pair);
                 const int n0 = tn * 256 + half * 128;
-                if (row < p.M && n0 < p.N)
+                if (p.tma_store) {
+                    if (row0 < p.M && n0 < p.N) {
+                        tma_store_chunk(packed, n0, row0);
+                        if (n0 + 64 < p.N) tma_store_chunk(packed + 32, n0 + 64, row0);
+                    }
+                } else if (row < p.M && n0 < p.N) {
                     store_row<128>(p.y + static_cast<int64_t>(row) * p.ldy + n0, packed, p.N - n0,
                                    vec_ok);
+                }
             } else {
                 uint32_t packed[32];
 #pragma unroll
@@ -370,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(acc_empty);
+                if (lane == 0) mbar_arrive_cluster(acc_empty_pair);
                 const int n0 = tn * 128 + half * 64;
                 if (row < p.M) {
 #pragma unroll
@@ -379,11 +425,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                         hmax = fmaxf(hmax, fmaxf(fabsf(__bfloat162float(v.x)),
                                                  fabsf(__bfloat162float(v.y))));
                     }
+                }
+                if (p.tma_store) {
+                    if (row0 < p.M) tma_store_chunk(packed, n0, row0);
+                } else if (row < p.M) {
                     store_row<64>(p.y + static_cast<int64_t>(row) * p.ldy + n0, packed, 64, true);
                 }
             }
             acc_phase ^= 1u;
         }
+        if (lane == 0) bulk_wait_group0();  // this warp's output stores have completed
+        __syncwarp();
         if (kSwiglu) {
             const uint32_t b = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(hmax));
             if (lane == 0) red[ew] = __uint_as_float(b);
@@ -398,20 +450,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     tc_fence_before();
     __syncthreads();
+    if (*abort_flag) {
+        // after a timeout, give copies this CTA issued toward the peer's
+        // barriers time to land before the pair tears down
+        const unsigned long long t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 1000000ull) {
+        }
+    }
+    cluster_sync();  // no peer signal or paired MMA can still target this CTA
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc_pair(tmem, kTmemCols);
     }
 }
 
-}  // namespace
+using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                              const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                              const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-bool encode_codes_tmap(CUtensorMap *map, const void *codes, int64_t rows, int64_t K) {
-    using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeFn encode_fn() {
     static EncodeFn fn = nullptr;
     if (!fn) {
         void *ptr = nullptr;
@@ -419,9 +478,17 @@ bool encode_codes_tmap(CUtensorMap *map, const void *codes, int64_t rows, int64_
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
                 cudaSuccess ||
             q != cudaDriverEntryPointSuccess || !ptr)
-            return false;
+            return nullptr;
         fn = reinterpret_cast<EncodeFn>(ptr);
     }
+    return fn;
+}
+
+}  // namespace
+
+bool encode_codes_tmap(CUtensorMap *map, const void *codes, int64_t rows, int64_t K) {
+    EncodeFn fn = encode_fn();
+    if (!fn) return false;
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
     const cuuint32_t box[2] = {128, 128};
@@ -432,12 +499,46 @@ bool encode_codes_tmap(CUtensorMap *map, const void *codes, int64_t rows, int64_
     return r == CUDA_SUCCESS;
 }
 
+bool encode_sf_tmap(CUtensorMap *map, const void *sf, int64_t rows, int64_t K) {
+    EncodeFn fn = encode_fn();
+    if (!fn) return false;
+    // the swizzled scales as an array of 512-byte tiles (128 words each); a box
+    // is the 4 consecutive tiles of one K step
+    const int64_t tiles = (rows + 127) / 128 * (K / 64);
+    const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(tiles)};
+    const cuuint64_t strides[1] = {512};
+    const cuuint32_t box[2] = {128, 4};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(sf), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool encode_out_tmap(CUtensorMap *map, const void *y, int64_t rows, int64_t cols, int64_t ld) {
+    EncodeFn fn = encode_fn();
+    if (!fn || ld % 8 != 0 || (reinterpret_cast<uintptr_t>(y) & 15u)) return false;
+    // BF16 [rows, cols] with leading dimension ld; a box is 32 rows x 64 columns
+    // (128 bytes, 128-byte swizzled in shared memory)
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * 2)};
+    const cuuint32_t box[2] = {64, 32};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(y), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 cudaError_t launch_gemm_nvf4(const CUtensorMap &tmap_a, const CUtensorMap &tmap_b,
+                             const CUtensorMap &tmap_sfa, const CUtensorMap &tmap_sfb,
                              const GemmArgs &a, bool swiglu, int num_sms, int *grid_out,
                              cudaStream_t s) {
     Params p;
-    p.sfa = a.sfa;
-    p.sfb = a.sfb;
+    CUtensorMap tmap_y;
+    std::memset(&tmap_y, 0, sizeof(tmap_y));
+    const int64_t out_cols = swiglu ? a.N / 2 : a.N;
+    p.tma_store = encode_out_tmap(&tmap_y, a.y, a.M, out_cols, a.ldy) ? 1 : 0;
     p.s_enc_a = a.s_enc_a;
     p.s_enc_b = a.s_enc_b;
     p.y = static_cast<__nv_bfloat16 *>(a.y);
@@ -445,29 +546,32 @@ cudaError_t launch_gemm_nvf4(const CUtensorMap &tmap_a, const CUtensorMap &tmap_
     p.M = a.M;
     p.N = a.N;
     p.K = a.K;
-    p.tiles_m = (a.M + 127) / 128;
+    p.tiles_m = (a.M + 255) / 256;
     p.n_half = a.N / 2;
     p.tiles_n = swiglu ? p.n_half / 128 : (a.N + 255) / 256;
     p.sf_ktiles = a.K / 64;
     p.k_tiles = (p.sf_ktiles + 3) / 4;
-    p.sf_rowblocks_b = (a.N + 127) / 128;
     p.amax_partials = a.amax_partials;
     p.err = a.err;
     const int tiles = p.tiles_m * p.tiles_n;
-    int grid = tiles < num_sms ? tiles : num_sms;
-    if (grid < 1) grid = 1;
+    const int max_pairs = num_sms / 2;
+    int pairs = tiles < max_pairs ? tiles : max_pairs;
+    if (pairs < 1) pairs = 1;
+    const int grid = 2 * pairs;
     if (grid_out) *grid_out = grid;
     cudaError_t e;
     if (swiglu) {
         e = cudaFuncSetAttribute(gemm_nvf4_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kSmemBytes);
         if (e != cudaSuccess) return e;
-        gemm_nvf4_kernel<true><<<grid, kThreads, kSmemBytes, s>>>(tmap_a, tmap_b, p);
+        gemm_nvf4_kernel<true><<<grid, kThreads, kSmemBytes, s>>>(tmap_a, tmap_b, tmap_sfa, tmap_sfb,
+                                                                   tmap_y, p);
     } else {
         e = cudaFuncSetAttribute(gemm_nvf4_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kSmemBytes);
         if (e != cudaSuccess) return e;
-        gemm_nvf4_kernel<false><<<grid, kThreads, kSmemBytes, s>>>(tmap_a, tmap_b, p);
+        gemm_nvf4_kernel<false><<<grid, kThreads, kSmemBytes, s>>>(tmap_a, tmap_b, tmap_sfa, tmap_sfb,
+                                                                    tmap_y, p);
     }
     return cudaGetLastError();
 }

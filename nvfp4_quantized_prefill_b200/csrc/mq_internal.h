@@ -25,8 +25,6 @@ cudaError_t launch_quantize(const void *x, int64_t M, int64_t K, int64_t ldx,
 // ---- block-scaled GEMM (mq_gemm.cu) ------------------------------------------
 
 struct GemmArgs {
-    const uint8_t *sfa;       // swizzled scales of A (activation)
-    const uint8_t *sfb;       // swizzled scales of B (weight)
     const float *s_enc_a;     // device scalars
     const float *s_enc_b;
     void *y;                  // BF16 output
@@ -39,12 +37,18 @@ struct GemmArgs {
 // Launches the tcgen05 GEMM; *grid_out receives the CTA count (the number of
 // amax partials written in SwiGLU mode).
 cudaError_t launch_gemm_nvf4(const CUtensorMap &tmap_a, const CUtensorMap &tmap_b,
+                             const CUtensorMap &tmap_sfa, const CUtensorMap &tmap_sfb,
                              const GemmArgs &a, bool swiglu, int num_sms, int *grid_out,
                              cudaStream_t s);
 
 // Host-side tensor map over an [rows, K/2]-byte code matrix, 128 x 128-byte
 // boxes with 128-byte swizzle.
 bool encode_codes_tmap(CUtensorMap *map, const void *codes, int64_t rows, int64_t K);
+
+// Host-side tensor map over a swizzled scale buffer of an [rows, K] operand,
+// seen as consecutive 512-byte scale tiles; one box = the 4 tiles of a
+// 256-wide K step of one 128-row block.
+bool encode_sf_tmap(CUtensorMap *map, const void *sf, int64_t rows, int64_t K);
 
 // ---- BF16 decode (mq_decode.cu) ------------------------------------------------
 
