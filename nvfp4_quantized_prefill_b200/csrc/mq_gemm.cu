@@ -13,7 +13,8 @@
 //   warp 0       (both CTAs) TMA producer: this CTA's 128 A rows and 128 B
 //                rows of a 256-wide K step (128-byte swizzle), its A scale
 //                tiles and both B scale halves, into a 5-stage ring; every
-//                load completes on the even CTA's stage barrier.
+//                load completes on the even CTA's stage barriers (scale tiles
+//                on their own, so their TMEM copies overlap the operand loads).
 //   warp 1       (even CTA) MMA issuer: 4 paired MMAs (K = 64 each) per stage
 //                into a 128 x 256 FP32 accumulator in each CTA's TMEM.
 //   warps 2-3    (even CTA) scale copiers: tcgen05.cp of the stage's scale
@@ -53,12 +54,13 @@ constexpr uint32_t kBBytes = 128 * 128;          // this CTA's 128 B rows
 constexpr uint32_t kSfaBytes = 4 * 512;          // 4 scale tiles (K = 256) of the A rows
 constexpr uint32_t kSfbBytes = 2 * 4 * 512;      // both 128-row halves of the B tile
 constexpr uint32_t kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // 38912
-constexpr uint32_t kPairTxBytes = 2 * kStageBytes;                           // both CTAs
+constexpr uint32_t kPairTxAB = 2 * (kABytes + kBBytes);                      // both CTAs
+constexpr uint32_t kPairTxSF = 2 * (kSfaBytes + kSfbBytes);
 constexpr uint32_t kStageTileBytes = 32 * 128;    // epilogue staging: 32 rows x 64 bf16
 constexpr uint32_t kStagingBytes = 8 * kStageTileBytes;  // one per epilogue warp
 constexpr uint32_t kBarBytes = 256;
 constexpr uint32_t kSmemBytes = kStages * kStageBytes + kStagingBytes + kBarBytes + 1024;
-constexpr int kCopiers = MQ_GEMM_COPIERS;        // scale-copy warps (even CTA)
+constexpr int kCopiers = MQ_GEMM_COPIERS;        // scale-copy warps (0: the MMA thread copies)
 constexpr int kEpiWarp0 = 2 + kCopiers;          // first of 8 epilogue warps
 constexpr int kThreads = 32 * (kEpiWarp0 + 8);
 constexpr uint32_t kTmemCols = 512;
@@ -69,7 +71,7 @@ constexpr uint16_t kPairMask = 0x3;
 
 static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
 static_assert(kSfCol + kStages * kSfColsPerStage <= kTmemCols, "TMEM budget");
-static_assert((3 * kStages + 4) * 8 + 48 <= kBarBytes, "barrier area");
+static_assert((4 * kStages + 4) * 8 + 48 <= kBarBytes, "barrier area");
 
 struct Params {
     const float *s_enc_a;
@@ -146,7 +148,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes + kStagingBytes);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * kStages + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 4 * kStages + 4);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     float *red = reinterpret_cast<float *>(tmem_slot + 2);  // 8 floats
 
@@ -156,7 +158,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t bar0 = smem_u32(bars);             // full[s]  = bar0 + 8 s
     const uint32_t empty0 = bar0 + 8u * kStages;      // empty[s]
     const uint32_t sf_full0 = bar0 + 16u * kStages;   // sf_full[s]
-    const uint32_t acc_full = bar0 + 24u * kStages;
+    const uint32_t sfd_full0 = bar0 + 24u * kStages;  // scale tiles landed[s]
+    const uint32_t acc_full = bar0 + 32u * kStages;
     const uint32_t acc_empty = acc_full + 8u;
     const uint32_t drain_bar = acc_full + 16u;
     const uint32_t sf_drain_bar = acc_full + 24u;
@@ -166,12 +169,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int s = 0; s < kStages; ++s) {
             mbar_init(bar0 + 8u * s, 1);             // arrive.expect_tx of the even CTA
             mbar_init(empty0 + 8u * s, 1);           // MMA commit (to both CTAs)
-            mbar_init(sf_full0 + 8u * s, kCopiers);  // one commit per copier
+            mbar_init(sf_full0 + 8u * s, kCopiers > 0 ? kCopiers : 1);  // one commit per copier
+            mbar_init(sfd_full0 + 8u * s, 1);        // arrive.expect_tx of the even CTA
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 16);                    // 8 epilogue warps x 2 CTAs
         mbar_init(drain_bar, 1);
-        mbar_init(sf_drain_bar, kCopiers);
+        mbar_init(sf_drain_bar, kCopiers > 0 ? kCopiers : 1);
         *abort_flag = 0;
         fence_barrier_init();
         prefetch_tmap(&tmap_a);
@@ -190,74 +194,85 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int pair = static_cast<int>(blockIdx.x >> 1);
     const int npairs = static_cast<int>(gridDim.x >> 1);
 
+    // The producer, MMA and copier roles run their loops on all 32 lanes with
+    // warp-uniform state; one elected lane issues each TMA / tcgen05
+    // instruction (see the warp_* wrappers).
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            uint32_t armed = 0, armed_parity = 0;
-            bool ok = true;
-            for (int t = pair; t < num_tiles && ok; t += npairs) {
-                int tm, tn;
-                tile_coords(t, p.tiles_m, p.tiles_n, tm, tn);
-                // B rows of this CTA and the two 128-row scale blocks of the tile
-                int b_row, rb0, rb1;
-                if (kSwiglu) {
-                    rb0 = tn;                            // gate rows 128 tn ..
-                    rb1 = p.n_half / 128 + tn;           // matching up rows
-                    b_row = (rank == 0 ? rb0 : rb1) * 128;
-                } else {
-                    rb0 = 2 * tn;
-                    rb1 = 2 * tn + 1;
-                    b_row = tn * 256 + static_cast<int>(rank) * 128;
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t armed = 0, armed_parity = 0;
+        bool ok = true;
+        for (int t = pair; t < num_tiles && ok; t += npairs) {
+            int tm, tn;
+            tile_coords(t, p.tiles_m, p.tiles_n, tm, tn);
+            // B rows of this CTA and the two 128-row scale blocks of the tile
+            int b_row, rb0, rb1;
+            if (kSwiglu) {
+                rb0 = tn;                            // gate rows 128 tn ..
+                rb1 = p.n_half / 128 + tn;           // matching up rows
+                b_row = (rank == 0 ? rb0 : rb1) * 128;
+            } else {
+                rb0 = 2 * tn;
+                rb1 = 2 * tn + 1;
+                b_row = tn * 256 + static_cast<int>(rank) * 128;
+            }
+            const int a_row = tm * 256 + static_cast<int>(rank) * 128;
+            const int a_sf = (2 * tm + static_cast<int>(rank)) * p.sf_ktiles;
+            for (int kt = 0; kt < p.k_tiles; ++kt) {
+                if (!warp_mbar_wait(empty0 + 8u * stage, phase ^ 1u, abort_flag, p.err)) {
+                    ok = false;
+                    break;
                 }
-                const int a_row = tm * 256 + static_cast<int>(rank) * 128;
-                const int a_sf = (2 * tm + static_cast<int>(rank)) * p.sf_ktiles;
-                for (int kt = 0; kt < p.k_tiles; ++kt) {
-                    if (!mbar_wait(empty0 + 8u * stage, phase ^ 1u, abort_flag, p.err)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t full_local = bar0 + 8u * stage;
-                    const uint32_t full_pair = mapa_shared(full_local, 0);
-                    if (rank == 0) {
-                        mbar_arrive_expect_tx(full_local, kPairTxBytes);
-                        armed |= 1u << stage;
-                        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-                    }
-                    const uint32_t sA = smem0 + stage * kStageBytes;
-                    const uint32_t sB = sA + kABytes;
-                    const uint32_t sSFA = sB + kBBytes;
-                    const uint32_t sSFB = sSFA + kSfaBytes;
-                    tma_load_2d_pair(sA, &tmap_a, kt * 128, a_row, full_pair);
-                    tma_load_2d_pair(sB, &tmap_b, kt * 128, b_row, full_pair);
-                    tma_load_2d_pair(sSFA, &tmap_sfa, 0, a_sf + kt * 4, full_pair);
-                    tma_load_2d_pair(sSFB, &tmap_sfb, 0, rb0 * p.sf_ktiles + kt * 4, full_pair);
-                    tma_load_2d_pair(sSFB + 4u * 512u, &tmap_sfb, 0, rb1 * p.sf_ktiles + kt * 4,
-                                     full_pair);
-                    if (++stage == kStages) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                const uint32_t full_local = bar0 + 8u * stage;
+                const uint32_t full_pair = mapa_shared(full_local, 0);
+                const uint32_t sfd_local = sfd_full0 + 8u * stage;
+                const uint32_t sfd_pair = mapa_shared(sfd_local, 0);
+                if (rank == 0) {
+                    warp_arrive_expect_tx(sfd_local, kPairTxSF);
+                    warp_arrive_expect_tx(full_local, kPairTxAB);
+                    armed |= 1u << stage;
+                    armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+                }
+                const uint32_t sA = smem0 + stage * kStageBytes;
+                const uint32_t sB = sA + kABytes;
+                const uint32_t sSFA = sB + kBBytes;
+                const uint32_t sSFB = sSFA + kSfaBytes;
+                // the small scale tiles first, on their own barrier, so the
+                // scale copies into TMEM can start before the operands land
+                warp_tma_load_2d_pair(sSFA, &tmap_sfa, 0, a_sf + kt * 4, sfd_pair);
+                warp_tma_load_2d_pair(sSFB, &tmap_sfb, 0, rb0 * p.sf_ktiles + kt * 4, sfd_pair);
+                warp_tma_load_2d_pair(sSFB + 4u * 512u, &tmap_sfb, 0, rb1 * p.sf_ktiles + kt * 4,
+                                      sfd_pair);
+                warp_tma_load_2d_pair(sA, &tmap_a, kt * 128, a_row, full_pair);
+                warp_tma_load_2d_pair(sB, &tmap_b, kt * 128, b_row, full_pair);
+                if (++stage == kStages) {
+                    stage = 0;
+                    phase ^= 1u;
                 }
             }
-            // both CTAs' loads of every armed stage land before the pair may exit
-            for (int s = 0; s < kStages; ++s)
-                if (armed & (1u << s)) drain_wait(bar0 + 8u * s, (armed_parity >> s) & 1u, p.err);
         }
+        // both CTAs' loads of every armed stage land before the pair may exit
+        for (int s2 = 0; s2 < kStages; ++s2)
+            if (armed & (1u << s2)) {
+                drain_wait(sfd_full0 + 8u * s2, (armed_parity >> s2) & 1u, p.err);
+                drain_wait(bar0 + 8u * s2, (armed_parity >> s2) & 1u, p.err);
+            }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0 && rank == 0) {
+        if (rank == 0) {
             constexpr uint32_t idesc = idesc_nvf4(256, 256);
             int stage = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
             for (int t = pair; t < num_tiles && ok; t += npairs) {
-                if (!mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag, p.err)) break;
+                if (!warp_mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag, p.err)) break;
                 tc_fence_after();
                 for (int kt = 0; kt < p.k_tiles; ++kt) {
-                    // operands of both CTAs landed and the stage's scales are in TMEM
-                    if (!mbar_wait(sf_full0 + 8u * stage, phase, abort_flag, p.err)) {
+                    // the stage's scales are in TMEM and both CTAs' operands landed
+                    const uint32_t sf_bar = kCopiers > 0 ? sf_full0 : sfd_full0;
+                    if (!warp_mbar_wait(sf_bar + 8u * stage, phase, abort_flag, p.err) ||
+                        !warp_mbar_wait(bar0 + 8u * stage, phase, abort_flag, p.err)) {
                         ok = false;
                         break;
                     }
@@ -267,23 +282,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const uint32_t sB = sA + kABytes;
                     const uint32_t tsfa = tmem + kSfCol + stage * kSfColsPerStage;
                     const uint32_t tsfb = tsfa + 16u;
-                    for (int kb = 0; kb < natoms; ++kb) {
-                        tc_mma_nvf4_pair(tmem, sdesc_kmajor_sw128(sA + 32u * kb),
-                                         sdesc_kmajor_sw128(sB + 32u * kb), idesc, tsfa + 4u * kb,
-                                         tsfb + 8u * kb, (kt | kb) != 0 ? 1u : 0u);
+                    if (kCopiers == 0) {
+                        // in-thread copies: ordered before this thread's MMAs below
+                        const uint32_t sSFA = sB + kBBytes;
+                        const uint32_t sSFB = sSFA + kSfaBytes;
+                        for (int a = 0; a < natoms; ++a) {
+                            warp_cp_sf_pair(tsfa + 4u * a, sdesc_sf_tile(sSFA + 512u * a));
+                            warp_cp_sf_pair(tsfb + 8u * a, sdesc_sf_tile(sSFB + 512u * a));
+                            warp_cp_sf_pair(tsfb + 8u * a + 4u,
+                                            sdesc_sf_tile(sSFB + 4u * 512u + 512u * a));
+                        }
                     }
-                    tc_commit_pair_mc(empty0 + 8u * stage, kPairMask);  // frees both CTAs' stage
+                    for (int kb = 0; kb < natoms; ++kb) {
+                        warp_mma_nvf4_pair(tmem, sdesc_kmajor_sw128(sA + 32u * kb),
+                                           sdesc_kmajor_sw128(sB + 32u * kb), idesc, tsfa + 4u * kb,
+                                           tsfb + 8u * kb, (kt | kb) != 0 ? 1u : 0u);
+                    }
+                    warp_commit_pair_mc(empty0 + 8u * stage, kPairMask);  // frees both CTAs' stage
                     if (++stage == kStages) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
                 if (!ok) break;
-                tc_commit_pair_mc(acc_full, kPairMask);
+                warp_commit_pair_mc(acc_full, kPairMask);
                 acc_phase ^= 1u;
             }
-            // every MMA issued by this thread completes before TMEM is freed
-            tc_commit_pair(drain_bar);
+            // every MMA issued by this warp completes before TMEM is freed
+            warp_commit_pair(drain_bar);
             drain_wait(drain_bar, 0, p.err);
         }
     } else if (warp < kEpiWarp0) {
@@ -292,13 +318,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // scale tile (each CTA its own rows) and both B halves, into the
         // stage's TMEM scale slot of both CTAs, then arrives on sf_full[stage].
         const int cid = warp - 2;
-        if (lane == 0 && rank == 0) {
+        if (rank == 0) {
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
             for (int t = pair; t < num_tiles && ok; t += npairs) {
                 for (int kt = 0; kt < p.k_tiles; ++kt) {
-                    if (!mbar_wait(bar0 + 8u * stage, phase, abort_flag, p.err)) {
+                    if (!warp_mbar_wait(sfd_full0 + 8u * stage, phase, abort_flag, p.err)) {
                         ok = false;
                         break;
                     }
@@ -309,18 +335,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const uint32_t tsfa = tmem + kSfCol + stage * kSfColsPerStage;
                     const uint32_t tsfb = tsfa + 16u;
                     for (int a = cid; a < natoms; a += kCopiers) {
-                        tc_cp_sf_pair(tsfa + 4u * a, sdesc_sf_tile(sSFA + 512u * a));
-                        tc_cp_sf_pair(tsfb + 8u * a, sdesc_sf_tile(sSFB + 512u * a));
-                        tc_cp_sf_pair(tsfb + 8u * a + 4u, sdesc_sf_tile(sSFB + 4u * 512u + 512u * a));
+                        warp_cp_sf_pair(tsfa + 4u * a, sdesc_sf_tile(sSFA + 512u * a));
+                        warp_cp_sf_pair(tsfb + 8u * a, sdesc_sf_tile(sSFB + 512u * a));
+                        warp_cp_sf_pair(tsfb + 8u * a + 4u, sdesc_sf_tile(sSFB + 4u * 512u + 512u * a));
                     }
-                    tc_commit_pair(sf_full0 + 8u * stage);
+                    warp_commit_pair(sf_full0 + 8u * stage);
                     if (++stage == kStages) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
             }
-            tc_commit_pair(sf_drain_bar);
+            warp_commit_pair(sf_drain_bar);
             drain_wait(sf_drain_bar, 0, p.err);
         }
     } else {
