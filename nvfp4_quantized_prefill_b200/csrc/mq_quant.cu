@@ -80,81 +80,131 @@ __device__ __forceinline__ float e4m3_to_float(uint32_t b) {
     return __half2float(__half(h));
 }
 
-// Four pairs of non-negative floats -> 4 bytes of E2M1x2 (second of each pair
-// in the high nibble), round-to-nearest-even, saturating at 6.
-__device__ __forceinline__ uint32_t e2m1x8(const float (&a)[8]) {
-    uint32_t out;
-    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-        : "=r"(out)
-        : "f"(a[0]), "f"(a[1]), "f"(a[2]), "f"(a[3]), "f"(a[4]), "f"(a[5]), "f"(a[6]),
-          "f"(a[7]));
-    return out;
-}
-
 // Byte offset of the 4 scales (r, 4*cq .. 4*cq+3) in the swizzled layout.
 __device__ __forceinline__ uint64_t sf_word_offset(uint32_t r, uint32_t cq, uint32_t ctiles) {
     return (static_cast<uint64_t>(r >> 7) * ctiles + cq) * 512u + (r & 31u) * 16u +
            ((r >> 5) & 3u) * 4u;
 }
 
-// One warp quantizes one 256-element segment of a row per iteration: lane l
-// owns elements [8l, 8l+8), lanes 2j and 2j+1 form 16-block j.
+#ifndef MQ_QUANT_HW_SIGN
+#define MQ_QUANT_HW_SIGN 1
+#endif
+constexpr int kQuantUnroll = 2;
+
+// fp32(a / 6) for a non-negative finite BF16 value a, in three operations:
+// q0 = RN(a * RN(1/6)), r = RN(a - 6 q0) (exact by FMA), q = RN(r * RN(1/6) + q0).
+// Checked exhaustively against IEEE division for all 32640 non-negative finite
+// BF16 inputs.
+__device__ __forceinline__ float div6_bf16(float a) {
+    const float inv6 = 0.16666667163372039794921875f;  // RN(1/6)
+    const float q0 = __fmul_rn(a, inv6);
+    const float r = __fmaf_rn(-q0, 6.0f, a);
+    return __fmaf_rn(r, inv6, q0);
+}
+
+// Two E2M1 codes (lo in bits 3:0, hi in bits 7:4) of x * f, round-to-nearest-even,
+// saturating at 6, sign from x (the conversion keeps the sign of a product
+// that rounds to zero).
+__device__ __forceinline__ uint32_t e2m1x2_signed(float lo, float hi) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 b;\n\tcvt.rn.satfinite.e2m1x2.f32 b, %2, %1;\n\tcvt.u32.u8 %0, b;\n\t}"
+        : "=r"(out)
+        : "f"(lo), "f"(hi));
+    return out;
+}
+
+// One lane quantizes one 16-element block held in w[0..7] (two BF16 per word,
+// element 2j in the low half of w[j]).  ftab[b] = s_enc / dec(b) for every
+// non-negative E4M3 byte b (0 for b = 0).  Returns the 8 code bytes in (lo, hi)
+// and the block scale byte in *sb_out.
+__device__ __forceinline__ void quantize_block16(const uint32_t (&w)[8], float s_enc,
+                                                 const float *ftab, uint32_t &lo, uint32_t &hi,
+                                                 uint32_t &sb_out) {
+    const uint32_t m = 0x7FFF7FFFu;
+    uint32_t a = __vmaxu2(__vmaxu2(w[0] & m, w[1] & m), __vmaxu2(w[2] & m, w[3] & m));
+    a = __vmaxu2(a, __vmaxu2(__vmaxu2(w[4] & m, w[5] & m), __vmaxu2(w[6] & m, w[7] & m)));
+    const float amax_b = __uint_as_float(max(a & 0xFFFFu, a >> 16) << 16);
+    const float sbf = __fmul_rn(div6_bf16(amax_b), s_enc);
+    const uint32_t sb = __nv_cvt_float_to_fp8(sbf, __NV_SATFINITE, __NV_E4M3);
+    const float f = ftab[sb];  // = dec(sb) == 0 ? 0 : fp32(s_enc / dec(sb))
+    uint32_t byte[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float x0 = __uint_as_float(w[j] << 16);
+        const float x1 = __uint_as_float(w[j] & 0xFFFF0000u);
+#if MQ_QUANT_HW_SIGN
+        byte[j] = e2m1x2_signed(__fmul_rn(x0, f), __fmul_rn(x1, f));
+#else
+        byte[j] = e2m1x2_signed(fabsf(__fmul_rn(x0, f)), fabsf(__fmul_rn(x1, f))) |
+                  ((w[j] >> 12) & 0x8u) | ((w[j] >> 24) & 0x80u);
+#endif
+    }
+    lo = byte[0] | (byte[1] << 8) | (byte[2] << 16) | (byte[3] << 24);
+    hi = byte[4] | (byte[5] << 8) | (byte[6] << 16) | (byte[7] << 24);
+    sb_out = sb;
+}
+
+// Each warp quantizes 512-element row segments (lane l: 16-block l of the
+// segment, two 16-byte loads), kQuantUnroll segments per iteration with all
+// loads issued first.  Lanes 4t..4t+3 hold the 4 scales of one swizzled
+// 32-bit scale word.
 __global__ void __launch_bounds__(kThreads) quantize_kernel(
     const uint4 *__restrict__ x, uint32_t M, uint32_t K, uint64_t ldv,
-    const float *__restrict__ partials, int n_partials, uint32_t *__restrict__ codes,
+    const float *__restrict__ partials, int n_partials, uint2 *__restrict__ codes,
     uint8_t *__restrict__ sf, float *__restrict__ s_enc_out, uint32_t Mpad) {
     __shared__ float red[kThreads / 32];
-    float a = 0.0f;
-    for (int i = threadIdx.x; i < n_partials; i += kThreads) a = fmaxf(a, partials[i]);
-    const float amax = block_max(a, red);
+    __shared__ float ftab[128];
+    float amx = 0.0f;
+    for (int i = threadIdx.x; i < n_partials; i += kThreads) amx = fmaxf(amx, partials[i]);
+    const float amax = block_max(amx, red);
     float s_enc = __fdiv_rn(2688.0f, amax);
     if (amax == 0.0f || !isfinite(s_enc)) s_enc = 1.0f;
     if (blockIdx.x == 0 && threadIdx.x == 0) *s_enc_out = s_enc;
+    if (threadIdx.x < 128) {
+        const float dec = e4m3_to_float(threadIdx.x);
+        ftab[threadIdx.x] = dec == 0.0f ? 0.0f : __fdiv_rn(s_enc, dec);
+    }
+    __syncthreads();
 
     const uint32_t ctiles = K / 64u;
-    const uint32_t segs = (K + 255u) / 256u;
+    const uint32_t kblocks = K / 16u;
+    const uint32_t segs = (K + 511u) / 512u;
     const uint32_t total = M * segs;
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t nwarps = gridDim.x * (kThreads / 32);
-    for (uint32_t seg = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); seg < total;
-         seg += nwarps) {
-        const uint32_t r = seg / segs, s = seg - r * segs;
-        const uint32_t k0 = s * 256u + lane * 8u;
-        const bool active = k0 < K;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (active) v = ldg_v4(x + r * ldv + k0 / 8u);
-        uint32_t mb = absmax8_bits(v);
-        mb = max(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, 1));
-        const float amax_b = __uint_as_float(mb << 16);
-        const float sbf = __fmul_rn(__fdiv_rn(amax_b, 6.0f), s_enc);
-        const uint32_t sb = __nv_cvt_float_to_fp8(sbf, __NV_SATFINITE, __NV_E4M3);
-        const float dec = e4m3_to_float(sb);
-        const float f = dec == 0.0f ? 0.0f : __fdiv_rn(s_enc, dec);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        float mag[8];
-        uint32_t signs = 0;
+    const uint32_t warp_id = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    for (uint32_t base = warp_id; base < total; base += nwarps * kQuantUnroll) {
+        uint32_t w[kQuantUnroll][8];
+        uint32_t rr[kQuantUnroll], bb[kQuantUnroll];
+        bool act[kQuantUnroll];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const uint32_t bits = (w[e >> 1] >> ((e & 1) * 16)) & 0xFFFFu;
-            mag[e] = fabsf(__fmul_rn(__uint_as_float(bits << 16), f));
-            signs |= (bits >> 15) << (4 * e + 3);
+        for (int u = 0; u < kQuantUnroll; ++u) {
+            const uint32_t seg = base + u * nwarps;
+            const uint32_t r = seg / segs, sg = seg - r * segs;
+            rr[u] = r;
+            bb[u] = sg * 32u + lane;  // block index within the row
+            act[u] = seg < total && bb[u] < kblocks;
+            uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+            if (act[u]) {
+                const uint4 *px = x + r * ldv + bb[u] * 2u;
+                v0 = ldg_v4(px);
+                v1 = ldg_v4(px + 1);
+            }
+            w[u][0] = v0.x; w[u][1] = v0.y; w[u][2] = v0.z; w[u][3] = v0.w;
+            w[u][4] = v1.x; w[u][5] = v1.y; w[u][6] = v1.z; w[u][7] = v1.w;
         }
-        const uint32_t word = e2m1x8(mag) | signs;
-        // scales of 4 consecutive blocks: lanes 8t, 8t+2, 8t+4, 8t+6
-        const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sb, 2);
-        const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sb, 4);
-        const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sb, 6);
-        if (active) {
-            codes[(static_cast<uint64_t>(r) * K + k0) / 8u] = word;
-            if ((lane & 7u) == 0) {
-                const uint32_t cq = k0 / 64u;
-                *reinterpret_cast<uint32_t *>(sf + sf_word_offset(r, cq, ctiles)) =
-                    sb | (s1 << 8) | (s2 << 16) | (s3 << 24);
+#pragma unroll
+        for (int u = 0; u < kQuantUnroll; ++u) {
+            uint32_t lo, hi, sb;
+            quantize_block16(w[u], s_enc, ftab, lo, hi, sb);
+            const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sb, 1);
+            const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sb, 2);
+            const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sb, 3);
+            if (act[u]) {
+                codes[static_cast<uint64_t>(rr[u]) * kblocks + bb[u]] = make_uint2(lo, hi);
+                if ((lane & 3u) == 0)
+                    *reinterpret_cast<uint32_t *>(sf + sf_word_offset(rr[u], bb[u] / 4u, ctiles)) =
+                        sb | (s1 << 8) | (s2 << 16) | (s3 << 24);
             }
         }
     }
@@ -190,7 +240,7 @@ cudaError_t launch_amax(const void *x, int64_t M, int64_t K, int64_t ldx, float 
 cudaError_t launch_quantize(const void *x, int64_t M, int64_t K, int64_t ldx,
                             const float *partials, int n_partials, uint8_t *codes,
                             uint8_t *sf_swizzled, float *s_enc, int num_sms, cudaStream_t s) {
-    const int64_t segs = M * ((K + 255) / 256);
+    const int64_t segs = M * ((K + 511) / 512);
     int64_t g = (segs + (kThreads / 32) - 1) / (kThreads / 32);
     const int64_t cap = 8LL * num_sms;
     if (g > cap) g = cap;
@@ -198,7 +248,7 @@ cudaError_t launch_quantize(const void *x, int64_t M, int64_t K, int64_t ldx,
     const int64_t Mpad = (M + 127) / 128 * 128;
     quantize_kernel<<<static_cast<int>(g), kThreads, 0, s>>>(
         static_cast<const uint4 *>(x), static_cast<uint32_t>(M), static_cast<uint32_t>(K),
-        static_cast<uint64_t>(ldx / 8), partials, n_partials, reinterpret_cast<uint32_t *>(codes),
+        static_cast<uint64_t>(ldx / 8), partials, n_partials, reinterpret_cast<uint2 *>(codes),
         sf_swizzled, s_enc, static_cast<uint32_t>(Mpad));
     return cudaGetLastError();
 }
