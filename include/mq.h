@@ -208,7 +208,10 @@ mq_status mq_prefill_linear_nvfp4_noalloc(const mq_weight *w, const void *x_bf16
 
 /* BF16 decode linear on the handle's BF16 copy: y[m, n] = bf16( sum_k x[m,k]
  * w[n,k] ) with FP32 accumulation.  x (device) BF16 [M, K] contiguous, y
- * (device) BF16 [M, N] contiguous.  Any M >= 1; meant for M <= 8. */
+ * (device) BF16 [M, N] contiguous.  Any M >= 1; meant for M <= 8.  For small
+ * N the K range is split across CTAs whose partial sums live in scratch inside
+ * the handle, so decode calls on the same handle must not overlap on the GPU
+ * (same stream, or ordered streams). */
 mq_status mq_decode_linear_bf16(const mq_weight *w, const void *x_bf16, int64_t M, void *y_bf16,
                                 cudaStream_t stream);
 

@@ -29,6 +29,7 @@ struct mq_weight {
     uint8_t *sf;         // swizzled scales, mq_sf_bytes(N, K)
     float *s_enc;        // device scalar
     float *partials;     // MQ_AMAX_PARTIALS_MAX floats (pack-time scratch)
+    void *decode_scratch; // K-slice partial sums + counters of the decode path
     CUtensorMap tmap;    // TMA map over the codes
     CUtensorMap tmap_sf; // TMA map over the swizzled scales
 };
@@ -225,7 +226,8 @@ mq_status mq_weight_pack(const void *w_bf16, int64_t N, int64_t K, cudaStream_t 
     const size_t b_codes = align256(static_cast<size_t>(N) * (K / 2));
     const size_t b_sf = align256(mq_sf_bytes(N, K));
     const size_t b_part = align256(sizeof(float) * MQ_AMAX_PARTIALS_MAX);
-    const size_t total = b_bf16 + b_codes + b_sf + b_part + 256;
+    const size_t b_dec = align256(mq::decode_scratch_bytes(N, K, d->num_sms));
+    const size_t total = b_bf16 + b_codes + b_sf + b_part + 256 + b_dec;
     if (cudaMalloc(&w->base, total) != cudaSuccess) {
         cudaGetLastError();
         delete w;
@@ -237,9 +239,12 @@ mq_status mq_weight_pack(const void *w_bf16, int64_t N, int64_t K, cudaStream_t 
     w->sf = w->codes + b_codes;
     w->partials = reinterpret_cast<float *>(w->sf + b_sf);
     w->s_enc = reinterpret_cast<float *>(w->sf + b_sf + b_part);
+    w->decode_scratch = b_dec ? static_cast<void *>(w->sf + b_sf + b_part + 256) : nullptr;
     st = MQ_OK;
-    if (cudaMemcpyAsync(w->bf16, w_bf16, static_cast<size_t>(N) * K * 2, cudaMemcpyDeviceToDevice,
-                        stream) != cudaSuccess)
+    if (b_dec && cudaMemsetAsync(w->decode_scratch, 0, b_dec, stream) != cudaSuccess)
+        st = MQ_ERR_CUDA;
+    if (st == MQ_OK && cudaMemcpyAsync(w->bf16, w_bf16, static_cast<size_t>(N) * K * 2,
+                                       cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
         st = MQ_ERR_CUDA;
     if (st == MQ_OK)
         st = quantize_impl(d, w->bf16, N, K, K, w->codes, w->sf, w->s_enc, nullptr, 0, w->partials,
@@ -471,8 +476,8 @@ mq_status mq_decode_linear_bf16(const mq_weight *w, const void *x_bf16, int64_t 
     DeviceInfo *d = nullptr;
     st = device_info(&d);
     if (st != MQ_OK) return st;
-    (void)d;
-    return cuda_status(mq::launch_decode(x_bf16, M, w->bf16, w->N, w->K, y_bf16, stream));
+    return cuda_status(mq::launch_decode(x_bf16, M, w->bf16, w->N, w->K, y_bf16, w->decode_scratch,
+                                         d->num_sms, stream));
 }
 
 }  // extern "C"

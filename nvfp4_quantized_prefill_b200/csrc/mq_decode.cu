@@ -5,15 +5,18 @@
 // the same weight handle that feeds the NVFP4 prefill GEMM keeps a BF16 copy
 // for this path, so the phase switch costs nothing.
 //
-// The op is bound by streaming W from HBM once (2 N K bytes).  Each CTA owns
-// 16 rows of W and its 8 warps split K; a warp reads, per step, 64 contiguous
-// bytes of each of its 16 rows (16-byte vector loads) plus the matching 64
-// bytes of each X row, and feeds them to two m16n8k16 BF16 MMAs (FP32
-// accumulate) with W rows as the M dimension and up to 8 X rows as N.  Both
-// fragments take the same K permutation (the 8 elements a thread loads), so no
-// shuffles or shared-memory staging are needed; for 8 tokens the tensor core
-// does the 8 FMAs per weight element that would otherwise saturate the FP32
-// pipes.  The cross-warp sum goes through shared memory.
+// The op is bound by streaming W from HBM once (2 N K bytes).  Work unit: 16
+// rows of W x one K slice.  A CTA (8 warps) owns one unit and its warps split
+// the slice; per step a warp reads 64 contiguous bytes of each of its 16 rows
+// (16-byte vector loads) plus the matching 64 bytes of each X row and feeds
+// two m16n8k16 BF16 MMAs (FP32 accumulate) with W rows as the M dimension and
+// up to 8 X rows as N.  Both fragments take the same K permutation (the 8
+// elements a thread loads), so no shuffles or staging are needed; for 8 tokens
+// the tensor core does the 8 FMAs per weight element that would otherwise
+// load the FP32 pipes.  K is split into S slices so that there are enough
+// units to balance the SMs; the last CTA of a row group to finish (an atomic
+// counter, reset by that CTA) adds the S partial sums in slice order --
+// deterministically -- and writes BF16.
 #include <cuda_bf16.h>
 
 #include "mq_internal.h"
@@ -24,6 +27,7 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kRows = 16;
+constexpr int kUnroll = 8;
 
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                                uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -36,15 +40,22 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
 
 __global__ void __launch_bounds__(kWarps * 32) decode_kernel(const uint4 *__restrict__ x, int M,
                                                              const uint4 *__restrict__ w, int N,
-                                                             int K, __nv_bfloat16 *__restrict__ y) {
+                                                             int K, int S,
+                                                             __nv_bfloat16 *__restrict__ y,
+                                                             float *__restrict__ partials,
+                                                             unsigned *__restrict__ counters) {
     __shared__ float part[kWarps][128];
+    __shared__ int last;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t4 = lane & 3;
-    const int n0 = blockIdx.x * kRows;
-    const int vpr = K / 8;               // 16-byte vectors per row
-    const int steps = K / 32;            // 32 K-elements per step (2 MMAs)
-    const int s0 = static_cast<int>(static_cast<int64_t>(steps) * warp / kWarps);
-    const int s1 = static_cast<int>(static_cast<int64_t>(steps) * (warp + 1) / kWarps);
+    const int group = blockIdx.x / S, slice = blockIdx.x - group * S;
+    const int n0 = group * kRows;
+    const int vpr = K / 8;                       // 16-byte vectors per row
+    const int steps = K / 32;                    // 32 K-elements per step (2 MMAs)
+    const int sl0 = static_cast<int>(static_cast<int64_t>(steps) * slice / S);
+    const int sl1 = static_cast<int>(static_cast<int64_t>(steps) * (slice + 1) / S);
+    const int s0 = sl0 + (sl1 - sl0) * warp / kWarps;
+    const int s1 = sl0 + (sl1 - sl0) * (warp + 1) / kWarps;
     const bool ra = n0 + g < N, rb = n0 + g + 8 < N, rx = g < M;
     const uint4 *wa = w + static_cast<int64_t>(ra ? n0 + g : 0) * vpr + t4;
     const uint4 *wb = w + static_cast<int64_t>(rb ? n0 + g + 8 : 0) * vpr + t4;
@@ -52,16 +63,16 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(const uint4 *__rest
     const uint4 z = make_uint4(0, 0, 0, 0);
     float c[4] = {0.f, 0.f, 0.f, 0.f};
     int s = s0;
-    for (; s + 4 <= s1; s += 4) {
-        uint4 va[4], vb[4], vx[4];
+    for (; s + kUnroll <= s1; s += kUnroll) {
+        uint4 va[kUnroll], vb[kUnroll], vx[kUnroll];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < kUnroll; ++u) {
             va[u] = ra ? __ldg(wa + (s + u) * 4) : z;
             vb[u] = rb ? __ldg(wb + (s + u) * 4) : z;
             vx[u] = rx ? __ldg(xr + (s + u) * 4) : z;
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < kUnroll; ++u) {
             mma_bf16_16816(c, va[u].x, vb[u].x, va[u].y, vb[u].y, vx[u].x, vx[u].y);
             mma_bf16_16816(c, va[u].z, vb[u].z, va[u].w, vb[u].w, vx[u].z, vx[u].w);
         }
@@ -76,30 +87,68 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(const uint4 *__rest
 #pragma unroll
     for (int i = 0; i < 4; ++i) part[warp][lane * 4 + i] = c[i];
     __syncthreads();
-    if (threadIdx.x < 128) {
-        const int q = threadIdx.x;
-        float acc = 0.f;
+    // accumulator element q = 4 * lane' + i': W row g' (+8 for i' >= 2), X row 2 t4' + (i' & 1)
+    const int q = threadIdx.x;  // one accumulator element per thread (first 128)
+    if (q >= 128) return;
+    float acc = 0.f;
 #pragma unroll
-        for (int i = 0; i < kWarps; ++i) acc += part[i][q];
-        // accumulator element q = 4 * lane' + i': row g' (+8 for i' >= 2), col 2 t4' + (i' & 1)
-        const int lq = q >> 2, iq = q & 3;
-        const int wrow = n0 + (lq >> 2) + ((iq >> 1) << 3);
-        const int m = 2 * (lq & 3) + (iq & 1);
+    for (int i = 0; i < kWarps; ++i) acc += part[i][q];
+    const int lq = q >> 2, iq = q & 3;
+    const int wrow = n0 + (lq >> 2) + ((iq >> 1) << 3);
+    const int m = 2 * (lq & 3) + (iq & 1);
+    if (S == 1) {
         if (m < M && wrow < N) y[static_cast<int64_t>(m) * N + wrow] = __float2bfloat16_rn(acc);
+        return;
     }
+    float *mine = partials + (static_cast<int64_t>(group) * S + slice) * 128;
+    mine[q] = acc;
+    __threadfence();
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (threadIdx.x == 0) last = (atomicAdd(&counters[group], 1u) == static_cast<unsigned>(S - 1));
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (!last) return;
+    __threadfence();
+    float sum = 0.f;
+    for (int k = 0; k < S; ++k)
+        sum += __ldcg(partials + (static_cast<int64_t>(group) * S + k) * 128 + q);
+    if (m < M && wrow < N) y[static_cast<int64_t>(m) * N + wrow] = __float2bfloat16_rn(sum);
+    if (threadIdx.x == 0) counters[group] = 0u;  // ready for the next call
 }
 
 }  // namespace
 
+int decode_slices(int64_t N, int64_t K, int num_sms) {
+    const int64_t groups = (N + kRows - 1) / kRows;
+    if (groups >= 2LL * num_sms) return 1;               // enough row groups to balance
+    int64_t S = (2LL * num_sms + groups - 1) / groups;   // >= 2 CTAs per SM
+    const int64_t max_s = K / 512 > 0 ? K / 512 : 1;     // keep >= 16 steps per slice
+    if (S > max_s) S = max_s;
+    if (S > 16) S = 16;
+    if (S < 1) S = 1;
+    return static_cast<int>(S);
+}
+
+size_t decode_scratch_bytes(int64_t N, int64_t K, int num_sms) {
+    const int S = decode_slices(N, K, num_sms);
+    if (S == 1) return 0;
+    const int64_t groups = (N + kRows - 1) / kRows;
+    return static_cast<size_t>(groups) * (S * 128 * sizeof(float) + sizeof(unsigned));
+}
+
 cudaError_t launch_decode(const void *x, int64_t M, const void *w, int64_t N, int64_t K, void *y,
-                          cudaStream_t s) {
-    const int grid = static_cast<int>((N + kRows - 1) / kRows);
+                          void *scratch, int num_sms, cudaStream_t s) {
+    const int S = decode_slices(N, K, num_sms);
+    const int64_t groups = (N + kRows - 1) / kRows;
+    float *partials = static_cast<float *>(scratch);
+    unsigned *counters =
+        S > 1 ? reinterpret_cast<unsigned *>(partials + groups * S * 128) : nullptr;
+    const int grid = static_cast<int>(groups * S);
     for (int64_t m0 = 0; m0 < M; m0 += 8) {
         const int mg = static_cast<int>(M - m0 < 8 ? M - m0 : 8);
         decode_kernel<<<grid, kWarps * 32, 0, s>>>(
             static_cast<const uint4 *>(x) + m0 * (K / 8), mg, static_cast<const uint4 *>(w),
-            static_cast<int>(N), static_cast<int>(K),
-            static_cast<__nv_bfloat16 *>(y) + m0 * N);
+            static_cast<int>(N), static_cast<int>(K), S, static_cast<__nv_bfloat16 *>(y) + m0 * N,
+            partials, counters);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

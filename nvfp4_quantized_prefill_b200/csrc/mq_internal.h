@@ -52,7 +52,14 @@ bool encode_sf_tmap(CUtensorMap *map, const void *sf, int64_t rows, int64_t K);
 
 // ---- BF16 decode (mq_decode.cu) ------------------------------------------------
 
+// Number of K slices the decode splits an [N, K] weight into, and the bytes of
+// per-weight scratch it needs for them (0 when S = 1): S x 128 FP32 partial
+// sums and one counter per 16-row group; the counters must start at zero and
+// are left at zero by every launch.
+int decode_slices(int64_t N, int64_t K, int num_sms);
+size_t decode_scratch_bytes(int64_t N, int64_t K, int num_sms);
+
 cudaError_t launch_decode(const void *x, int64_t M, const void *w, int64_t N, int64_t K,
-                          void *y, cudaStream_t s);
+                          void *y, void *scratch, int num_sms, cudaStream_t s);
 
 }  // namespace mq
