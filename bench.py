@@ -1,14 +1,17 @@
 """Benchmark of the prefill-phase NVFP4 linear layer (Mix-Quant hot path).
 
-One step = one pass of the hot path over one batch of synthetic input: for
-each projection of the workload, tensor amax -> NVFP4 quantize -> block-scaled
-GEMM (the prefill phase), then the BF16 decode linear at M = 1 on the same
-weight handles (the phase switch).
+One step = one pass of the hot path over one batch of synthetic input: the
+prefill phase of the workload's projections -- per activation: tensor amax ->
+NVFP4 quantize -> block-scaled tcgen05 GEMM (with the SwiGLU epilogue and the
+quantize of h between gate/up and down for MLP workloads) -- then the BF16
+decode linear at M = 1 on the same weight handles (the phase switch).
 
-Reported metric: prefill linear TFLOP/s including activation quantization,
-2*M*N*K summed over projections / (t_amax + t_quant + t_gemm), plus its
-fraction of the dense FP4 peak.  Timed with CUDA events on the launching
-stream, L2 flushed (256 MiB write) between steps outside the timed intervals.
+Metric: prefill linear TFLOP/s including activation quantization,
+sum(2 M N K) / (t_amax + t_quant + t_gemm [+ t_quant(h)]), and its fraction of
+the dense FP4 peak.  Timed with CUDA events on the launching stream; between
+steps, outside the timed intervals, the L2 is flushed by writing one 256 MiB
+buffer and then reading another, so no dirty lines are left for the next
+kernel to write back.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference ...   (the CPU oracle, bounded sample)
@@ -19,6 +22,7 @@ needs no exchange); value = work of all ranks / max-over-ranks time.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -38,6 +42,9 @@ METRIC = "prefill linear TFLOPS (NVFP4 incl. act-quant) and % of B200 dense FP4 
 CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+GEMM_SOURCES = ["nvfp4_quantized_prefill_b200/csrc/mq_gemm.cu",
+                "nvfp4_quantized_prefill_b200/csrc/mq_ptx.cuh"]
+COUNTERS = os.path.join(ROOT, "profiles", "counters.json")
 
 
 def peaks():
@@ -48,6 +55,29 @@ def peaks():
                 "bf16_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
                 "source": "measured"}
     return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+def gemm_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in GEMM_SOURCES:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload_key: str):
+    """DRAM bytes (read + write) per GEMM launch from the committed ncu summary,
+    only if it was taken on the GEMM source as it is now.  Returns
+    (mean bytes over the captured launches, their names) or (None, None)."""
+    try:
+        d = json.load(open(COUNTERS))
+    except Exception:
+        return None, None
+    if d.get("gemm_source_hash") != gemm_source_hash():
+        return None, None
+    per = d.get("gemm_dram_bytes_per_launch", {}).get(workload_key)
+    if not per:
+        return None, None
+    return sum(per.values()) / len(per), sorted(per)
 
 
 class ClockSampler:
@@ -86,8 +116,9 @@ class ClockSampler:
             return None
         if not rows:
             return None
-        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        num = lambda v: v.strip().replace(".", "", 1).isdigit()
+        sm = [float(r[1]) for r in rows if num(r[1])]
+        mx = [float(r[2]) for r in rows if num(r[2])]
         reasons = set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for r in rows:
@@ -99,7 +130,7 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
-def dist_setup(n_gpus: int):
+def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -118,20 +149,22 @@ def barrier(world):
         torch.distributed.barrier()
 
 
-def max_over_ranks(v: float, world: int) -> float:
+def reduce_over_ranks(v: float, world: int, op: str) -> float:
+    """MAX or SUM of a host float over the ranks (NCCL: via the GPU; gloo: CPU)."""
     if world == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=getattr(torch.distributed.ReduceOp, op))
     return float(t.item())
 
 
-def sum_over_ranks(v: float, world: int) -> float:
-    if world == 1:
-        return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
-    return float(t.item())
+def aggregate(flops_local: float, prefill_ms_local: float, world: int):
+    """Whole-job throughput of independent replicas: the work of all ranks over
+    the slowest rank's time.  Returns (tflops, max_ms, total_flops)."""
+    max_ms = reduce_over_ranks(prefill_ms_local, world, "MAX")
+    total = reduce_over_ranks(flops_local, world, "SUM")
+    return total / (max_ms * 1e-3) / 1e12, max_ms, total
 
 
 # ---------------------------------------------------------------------------
@@ -169,127 +202,271 @@ def oracle_sample(xs, wq, rows_per_linear: int):
 # GPU leg
 # ---------------------------------------------------------------------------
 
+class Prefill:
+    """Device buffers and the launch sequence of one workload's prefill."""
+
+    def __init__(self, wl, mq, dev):
+        self.wl, self.mq, self.dev = wl, mq, dev
+        ws = workloads.layer_weights(wl, device=str(dev))
+        self.ws = ws
+        self.W = [mq.Weight(w) for w in ws]
+        M = wl.M
+        self.M = M
+        u8, f32, bf = torch.uint8, torch.float32, torch.bfloat16
+
+        def qbuf(K):
+            return dict(codes=torch.empty(M, K // 2, dtype=u8, device=dev),
+                        sf=torch.empty(mq.mq_sf_bytes(M, K), dtype=u8, device=dev),
+                        s=torch.empty(1, dtype=f32, device=dev),
+                        part=torch.empty(mq.MQ_AMAX_PARTIALS_MAX, dtype=f32, device=dev))
+
+        self.ops = []    # list of (name, callable) kernel launches, in order
+        self.flops = 0.0
+        if wl.swiglu:
+            # pairs of (gate_up, down)
+            self.xs = []
+            for i in range(0, len(self.W), 2):
+                Wgu, Wd = self.W[i], self.W[i + 1]
+                I = Wgu.N // 2
+                x = workloads.layer_activation(wl, Wgu.K, i, device=str(dev))
+                self.xs.append(x)
+                qx, qh = qbuf(Wgu.K), qbuf(I)
+                h = torch.empty(M, I, dtype=bf, device=dev)
+                y = torch.empty(M, Wd.N, dtype=bf, device=dev)
+                self._add_quant(f"amax+quant x{i}", x, Wgu.K, qx)
+                self.ops.append((f"gemm {wl.linears[i].name}+swiglu", "gemm",
+                                 lambda st, qx=qx, Wgu=Wgu, h=h, qh=qh: qh.__setitem__(
+                                     "n", mq.mq_gemm_nvfp4_swiglu(qx["codes"], qx["sf"], qx["s"], M,
+                                                                  Wgu.handle, h, qh["part"], st))))
+                self.ops.append((f"quant h{i}", "quant",
+                                 lambda st, h=h, qh=qh, I=I: mq.mq_quantize_nvfp4(
+                                     h, M, I, I, qh["codes"], qh["sf"], qh["s"],
+                                     amax_partials=qh["part"], n_partials=qh["n"], stream=st)))
+                self.ops.append((f"gemm {wl.linears[i + 1].name}", "gemm",
+                                 lambda st, qh=qh, Wd=Wd, y=y: mq.mq_gemm_nvfp4(
+                                     qh["codes"], qh["sf"], qh["s"], M, Wd.handle, y, Wd.N, st)))
+                self.flops += 2.0 * M * Wgu.N * Wgu.K + 2.0 * M * Wd.N * Wd.K
+        elif wl.chunks > 1:
+            # each chunk quantized once and used by every projection
+            K = self.W[0].K
+            self.xs = [workloads.layer_activation(wl, K, c, device=str(dev)) for c in range(wl.chunks)]
+            q = qbuf(K)
+            ys = [torch.empty(M, W.N, dtype=bf, device=dev) for W in self.W]
+            for c, x in enumerate(self.xs):
+                self._add_quant(f"amax+quant chunk{c}", x, K, q)
+                for W, y, lin in zip(self.W, ys, wl.linears):
+                    self.ops.append((f"gemm {lin.name} chunk{c}", "gemm",
+                                     lambda st, q=q, W=W, y=y: mq.mq_gemm_nvfp4(
+                                         q["codes"], q["sf"], q["s"], M, W.handle, y, W.N, st)))
+                    self.flops += 2.0 * M * W.N * W.K
+        else:
+            self.xs = []
+            for i, (W, lin) in enumerate(zip(self.W, wl.linears)):
+                x = workloads.layer_activation(wl, W.K, i, device=str(dev))
+                self.xs.append(x)
+                q = qbuf(W.K)
+                y = torch.empty(M, W.N, dtype=bf, device=dev)
+                self._add_quant(f"amax+quant x{i}", x, W.K, q)
+                self.ops.append((f"gemm {lin.name}", "gemm",
+                                 lambda st, q=q, W=W, y=y: mq.mq_gemm_nvfp4(
+                                     q["codes"], q["sf"], q["s"], M, W.handle, y, W.N, st)))
+                self.flops += 2.0 * M * W.N * W.K
+        # decode (phase switch) on every weight handle at M = 1
+        self.dec = []
+        xdec = self.xs[0][:1]
+        for W in self.W:
+            xd = xdec if W.K == xdec.shape[1] else torch.zeros(1, W.K, dtype=bf, device=dev)
+            yd = torch.empty(1, W.N, dtype=bf, device=dev)
+            self.dec.append(lambda st, W=W, xd=xd, yd=yd: mq.mq_decode_linear_bf16(
+                W.handle, xd, 1, yd, st))
+        self.decode_bytes = sum(2.0 * W.N * W.K + 2.0 * W.K + 2.0 * W.N for W in self.W)
+        self.launches = len(self.ops) + len(self.dec)   # one kernel per op / decode call
+
+    def _add_quant(self, name, x, K, q):
+        mq, M = self.mq, self.M
+
+        def amax(st):
+            q["n"] = mq.mq_tensor_amax(x, M, K, K, q["part"], st)
+
+        self.ops.append((name.replace("amax+quant", "amax"), "amax", amax))
+        self.ops.append((name.replace("amax+quant", "quant"), "quant",
+                         lambda st: mq.mq_quantize_nvfp4(x, M, K, K, q["codes"], q["sf"], q["s"],
+                                                         amax_partials=q["part"],
+                                                         n_partials=q["n"], stream=st)))
+
+    def run_prefill(self, st):
+        for _, _, f in self.ops:
+            f(st)
+
+    def run_decode(self, st):
+        for f in self.dec:
+            f(st)
+
+    def free(self):
+        for W in self.W:
+            W.free()
+
+
 def run_gpu(args, wl, world, rank):
     from nvfp4_quantized_prefill_b200 import binding as mq
     mq.lib()
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
     pk = peaks()
+    P = Prefill(wl, mq, dev)
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(256 << 20, dtype=torch.uint8, device=dev)
+    sink = torch.empty((), dtype=torch.int64, device=dev)
 
-    ws_cpu = workloads.layer_weights(wl)
-    xs_cpu = [workloads.layer_activation(wl, w.shape[1], i) for i, w in enumerate(ws_cpu)]
-    Ws = [mq.Weight(w.to(dev)) for w in ws_cpu]
-    xs = [x.to(dev) for x in xs_cpu]
-    M = wl.M
-    bufs = []
-    for W in Ws:
-        K = W.K
-        bufs.append(dict(
-            codes=torch.empty(M, K // 2, dtype=torch.uint8, device=dev),
-            sf=torch.empty(mq.mq_sf_bytes(M, K), dtype=torch.uint8, device=dev),
-            s=torch.empty(1, dtype=torch.float32, device=dev),
-            part=torch.empty(mq.MQ_AMAX_PARTIALS_MAX, dtype=torch.float32, device=dev),
-            y=torch.empty(M, W.N, dtype=torch.bfloat16, device=dev),
-            yd=torch.empty(1, W.N, dtype=torch.bfloat16, device=dev)))
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    flops = sum(2.0 * M * W.N * W.K for W in Ws)
-    gemm_flops = flops
-    decode_bytes = sum(2.0 * W.N * W.K + 2.0 * W.K + 2.0 * W.N for W in Ws)
-    launches_per_step = 3 * len(Ws) + len(Ws)
+    def flush():
+        flush_w.zero_()
+        torch.sum(flush_r, dim=0, dtype=torch.int64, out=sink)
+
+    nop = len(P.ops)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
 
     def step(evs):
-        """evs: list of events, 4 per projection (start, after amax, after
-        quantize, after gemm) + 2 for decode (start, end)."""
-        i = 0
-        for W, x, b in zip(Ws, xs, bufs):
-            evs[i].record(stream)
-            n = mq.mq_tensor_amax(x, M, W.K, W.K, b["part"], stream)
+        evs[0].record(stream)
+        for i, (_, _, f) in enumerate(P.ops):
+            f(stream)
             evs[i + 1].record(stream)
-            mq.mq_quantize_nvfp4(x, M, W.K, W.K, b["codes"], b["sf"], b["s"],
-                                 amax_partials=b["part"], n_partials=n, stream=stream)
-            evs[i + 2].record(stream)
-            mq.mq_gemm_nvfp4(b["codes"], b["sf"], b["s"], M, W.handle, b["y"], W.N, stream)
-            evs[i + 3].record(stream)
-            i += 4
-        evs[i].record(stream)
-        for W, x, b in zip(Ws, xs, bufs):
-            mq.mq_decode_linear_bf16(W.handle, x[:1], 1, b["yd"], stream)
-        evs[i + 1].record(stream)
+        P.run_decode(stream)
+        evs[nop + 1].record(stream)
 
-    nev = 4 * len(Ws) + 2
     for _ in range(args.warmup):
-        flush.zero_()
-        step([torch.cuda.Event(enable_timing=True) for _ in range(nev)])
+        flush()
+        step([ev() for _ in range(nop + 2)])
     torch.cuda.synchronize()
-    st = mq.mq_check(stream)
-    if st != 0:
-        raise RuntimeError(f"device error during warm-up: {mq.STATUS.get(st)}")
+    if mq.mq_check(stream) != 0:
+        raise RuntimeError("device error during warm-up")
 
-    all_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
+    all_evs = [[ev() for _ in range(nop + 2)] for _ in range(args.steps)]
     clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
     barrier(world)
     torch.cuda.synchronize()
     with clocks:
         time.sleep(0.3)
         for k in range(args.steps):
-            flush.zero_()
+            flush()
             step(all_evs[k])
         torch.cuda.synchronize()
     barrier(world)
-    st = mq.mq_check(stream)
-    if st != 0:
-        raise RuntimeError(f"device error during timing: {mq.STATUS.get(st)}")
+    if mq.mq_check(stream) != 0:
+        raise RuntimeError("device error during timing")
 
-    t_amax = t_quant = t_gemm = t_dec = t_step = 0.0
+    per_kind = {"amax": 0.0, "quant": 0.0, "gemm": 0.0}
+    per_op = [0.0] * nop
+    t_dec = t_step = 0.0
     for evs in all_evs:
-        i = 0
-        for _ in Ws:
-            t_amax += evs[i].elapsed_time(evs[i + 1])
-            t_quant += evs[i + 1].elapsed_time(evs[i + 2])
-            t_gemm += evs[i + 2].elapsed_time(evs[i + 3])
-            i += 4
-        t_dec += evs[i].elapsed_time(evs[i + 1])
-        t_step += evs[0].elapsed_time(evs[i + 1])
+        for i, (_, kind, _) in enumerate(P.ops):
+            d = evs[i].elapsed_time(evs[i + 1])
+            per_kind[kind] += d
+            per_op[i] += d
+        t_dec += evs[nop].elapsed_time(evs[nop + 1])
+        t_step += evs[0].elapsed_time(evs[nop + 1])
     K_ = args.steps
-    t_prefill_ms = (t_amax + t_quant + t_gemm) / K_
-    t_prefill_max = max_over_ranks(t_prefill_ms, world)
-    t_step_max = max_over_ranks(t_step / K_, world)
-    total_flops = sum_over_ranks(flops, world)
-    value = total_flops / (t_prefill_max * 1e-3) / 1e12
-    gemm_ms = t_gemm / K_
+    t_prefill_ms = sum(per_kind.values()) / K_
+    value, t_prefill_max, total_flops = aggregate(P.flops, t_prefill_ms, world)
+    t_step_max = reduce_over_ranks(t_step / K_, world, "MAX")
+    gemm_ms = per_kind["gemm"] / K_
+    n_gemm = sum(1 for o in P.ops if o[1] == "gemm")
     fp4_peak = pk["bf16"] * FP4_OVER_BF16
-    achieved = gemm_flops / (gemm_ms * 1e-3) / 1e12
+    achieved = P.flops / (gemm_ms * 1e-3) / 1e12
+
+    # ---- CUDA-graph replay of the same prefill: a launch-overhead cross-check
+    graph_ms = None
+    try:
+        g = torch.cuda.CUDAGraph()
+        s2 = torch.cuda.Stream()
+        s2.wait_stream(stream)
+        with torch.cuda.stream(s2):
+            with torch.cuda.graph(g, stream=s2):
+                P.run_prefill(s2)
+        torch.cuda.synchronize()
+        gt = []
+        for _ in range(max(3, min(args.steps, 10))):
+            flush()
+            a, b = ev(), ev()
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+            gt.append(a.elapsed_time(b))
+        graph_ms = statistics.median(gt)
+        del g
+    except Exception as e:  # report, do not hide
+        graph_ms = f"unavailable: {type(e).__name__}: {e}"[:200]
+    if mq.mq_check(stream) != 0:
+        raise RuntimeError("device error during graph replay")
+
+    # ---- the same-shape BF16 path (cuBLAS through torch.matmul): comparator only
+    bf16_ms = None
+    try:
+        def bf16_prefill():
+            if wl.swiglu:
+                for i in range(0, len(P.ws), 2):
+                    gu = torch.matmul(P.xs[i // 2], P.ws[i].t())
+                    I = gu.shape[1] // 2
+                    h = torch.nn.functional.silu(gu[:, :I]) * gu[:, I:]
+                    torch.matmul(h, P.ws[i + 1].t())
+            elif wl.chunks > 1:
+                for x in P.xs:
+                    for w in P.ws:
+                        torch.matmul(x, w.t())
+            else:
+                for x, w in zip(P.xs, P.ws):
+                    torch.matmul(x, w.t())
+        bf16_prefill()
+        bt = []
+        for _ in range(max(3, min(args.steps, 10))):
+            flush()
+            a, b = ev(), ev()
+            a.record(stream)
+            bf16_prefill()
+            b.record(stream)
+            torch.cuda.synchronize()
+            bt.append(a.elapsed_time(b))
+        bf16_ms = statistics.median(bt)
+    except Exception as e:
+        bf16_ms = None
 
     # ---- end to end through the public call: pinned host X -> device, prefill
     # linear (amax + quantize + GEMM inside), result back to pinned host memory
-    xs_h = [x.pin_memory() for x in xs_cpu]
-    ys_h = [torch.empty(M, W.N, dtype=torch.bfloat16).pin_memory() for W in Ws]
-    xs_d = [torch.empty_like(x) for x in xs]
-    wsb = max(mq.mq_workspace_bytes(M, W.K) for W in Ws)
-    wsp = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    e2e = None
+    if not wl.swiglu and wl.chunks == 1:
+        M = wl.M
+        xs_h = [x.cpu().pin_memory() for x in P.xs]
+        ys_h = [torch.empty(M, W.N, dtype=torch.bfloat16).pin_memory() for W in P.W]
+        xs_d = [torch.empty_like(x) for x in P.xs]
+        ys_d = [torch.empty(M, W.N, dtype=torch.bfloat16, device=dev) for W in P.W]
+        wsb = max(mq.mq_workspace_bytes(M, W.K) for W in P.W)
+        wsp = torch.empty(wsb, dtype=torch.uint8, device=dev)
 
-    def e2e_step():
-        for W, xh, xd, b, yh in zip(Ws, xs_h, xs_d, bufs, ys_h):
-            xd.copy_(xh, non_blocking=True)
-            mq.mq_prefill_linear_nvfp4(W.handle, xd, M, b["y"], wsp, wsb, stream)
-            yh.copy_(b["y"], non_blocking=True)
+        def e2e_step():
+            for W, xh, xd, yd, yh in zip(P.W, xs_h, xs_d, ys_d, ys_h):
+                xd.copy_(xh, non_blocking=True)
+                mq.mq_prefill_linear_nvfp4(W.handle, xd, M, yd, wsp, wsb, stream)
+                yh.copy_(yd, non_blocking=True)
 
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2e_steps = max(2, min(args.steps, 10))
-    barrier(world)
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
-    h2d = sum(x.numel() * 2 for x in xs_cpu)
-    d2h = sum(M * W.N * 2 for W in Ws)
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        e0, e1 = ev(), ev()
+        n_e2e = max(2, min(args.steps, 10))
+        barrier(world)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = reduce_over_ranks(e0.elapsed_time(e1) / n_e2e, world, "MAX")
+        e2e = {"value": round(total_flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": sum(x.numel() * 2 for x in P.xs),
+               "d2h_bytes_per_step": sum(M * W.N * 2 for W in P.W),
+               "path": "mq_prefill_linear_nvfp4, pinned-host X in / Y out, per projection"}
 
+    traffic, traffic_launches = recorded_traffic(args.workload)
     clk = clocks.summary()
     out = {
         "metric": METRIC,
@@ -302,46 +479,50 @@ def run_gpu(args, wl, world, rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "nvfp4 (e2m1 + e4m3 block scales) x nvfp4 -> fp32 acc -> bf16",
-        "data": "synthetic (seeded, Llama-3-8B-shaped projections; random-init weights)",
+        "dtype": "nvfp4 (e2m1 codes, e4m3 per-16 scales, fp32 tensor scale) -> fp32 acc -> bf16",
+        "data": "synthetic (seeded recipe, random-init weights of the named shapes)",
         "config": {
             "workload": wl.name,
-            "tokens": M,
+            "workload_key": args.workload,
+            "tokens": wl.M * max(1, wl.chunks),
             "linears": [{"name": l.name, "N": l.N, "K": l.K} for l in wl.linears],
             "activations": wl.act,
             "seed": wl.seed,
-            "step": "per projection: tensor amax -> NVFP4 quantize -> block-scaled GEMM; "
-                    "then BF16 decode M=1 on the same weights",
-            "l2": "flushed between steps (256 MiB write, outside timed intervals)",
+            "step": "prefill (amax -> NVFP4 quantize -> tcgen05 block-scaled GEMM per "
+                    "activation) then BF16 decode M=1 on the same weight handles",
+            "l2": "flushed between steps: write 256 MiB, then read another 256 MiB "
+                  "(outside the timed intervals)",
             "parallelism": f"replicas x{world} (no exchange)",
         },
         "prefill_ms": round(t_prefill_max, 4),
-        "breakdown_ms": {"amax": round(t_amax / K_, 4), "quantize": round(t_quant / K_, 4),
-                         "gemm": round(gemm_ms, 4), "decode_m1": round(t_dec / K_, 4)},
-        "tokens_per_s": round(world * M / (t_prefill_max * 1e-3), 1),
+        "breakdown_ms": {k: round(v / K_, 4) for k, v in per_kind.items()},
+        "per_launch_ms": {P.ops[i][0]: round(per_op[i] / K_, 4) for i in range(nop)},
+        "decode_m1_ms": round(t_dec / K_, 4),
+        "decode_gbs": round(P.decode_bytes / (t_dec / K_ * 1e-3) / 1e9, 1),
+        "graph_prefill_ms": round(graph_ms, 4) if isinstance(graph_ms, float) else graph_ms,
+        "tokens_per_s": round(world * wl.M * max(1, wl.chunks) / (t_prefill_max * 1e-3), 1),
         "fp4_peak_frac": round(value / fp4_peak, 4),
         "gemm_only_tflops": round(achieved, 2),
-        "decode_gbs": round(decode_bytes / (t_dec / K_ * 1e-3) / 1e9, 1),
+        "bf16_cublas_ms": round(bf16_ms, 4) if bf16_ms else None,
+        "speedup_vs_bf16": round(bf16_ms / t_prefill_ms, 3) if bf16_ms else None,
         "roofline": {
-            "kernel": "gemm_nvf4_kernel (tcgen05 mxf4nvf4 block16)",
+            "kernel": "gemm_nvf4_kernel (tcgen05.mma.cta_group::2 kind::mxf4nvf4 block16)",
             "bound": "tensor",
             "achieved": round(achieved, 2),
             "peak": round(fp4_peak, 1),
             "peak_source": f"{pk['source']} bf16 burst {pk['bf16']} TF/s x {FP4_OVER_BF16} "
-                           "(nominal dense fp4/bf16 ratio)",
+                           "(nominal dense fp4/bf16 ratio), of measured",
             "unit": "TFLOP/s",
             "frac": round(achieved / fp4_peak, 4),
-            "traffic": None,
+            "traffic": traffic,
+            "traffic_launches": traffic_launches,
+            "launches_per_step": n_gemm,
         },
-        "e2e": {"value": round(total_flops / (e2e_ms * 1e-3) / 1e12, 3),
-                "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "path": "mq_prefill_linear_nvfp4 with pinned-host X in / Y out"},
-        "gpu_launches": launches_per_step * args.steps,
+        "e2e": e2e,
+        "gpu_launches": P.launches * args.steps,
         "clocks": clk,
     }
-    for W in Ws:
-        W.free()
-    return out, xs_cpu, ws_cpu
+    return out, P
 
 
 def main():
@@ -358,7 +539,6 @@ def main():
     wl = workloads.WORKLOADS[args.workload]
 
     if args.impl == "reference":
-        world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))
         if rank != 0:
             return
@@ -377,7 +557,7 @@ def main():
             "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": sum(times) / len(times) * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "int64 exact / fp64",
+            "scaling": "weak", "vs_baseline": None, "dtype": "int64 exact sum / fp64",
             "data": "synthetic", "config": {"workload": wl.name, "tokens": wl.M},
             "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": oracle.threads_used(),
                              "kind": "oracle",
@@ -387,16 +567,19 @@ def main():
                     "d2h_bytes_per_step": 0}}))
         return
 
-    world, rank, local = dist_setup(args.gpus)
-    out, xs_cpu, ws_cpu = run_gpu(args, wl, world, rank)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    world, rank, local = dist_setup()
+    out, P = run_gpu(args, wl, world, rank)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not wl.swiglu and wl.chunks == 1:
         import oracle
+        xs_cpu = [x.cpu() for x in P.xs]
+        ws_cpu = [w.cpu() for w in P.ws]
         fl, t = oracle_sample(xs_cpu, oracle_prepare(ws_cpu), args.cpu_rows)
         out["cpu_baseline"] = {"value": fl / t / 1e12, "unit": "TFLOP/s",
                                "cores": oracle.threads_used(), "kind": "oracle",
                                "sample": f"{args.cpu_rows} activation rows per projection "
                                          "(full-tensor amax, row quantize, exact GEMM); "
                                          f"{t:.1f} s"}
+    P.free()
     if rank == 0:
         print(json.dumps(out))
     if world > 1:

@@ -26,38 +26,47 @@ import torch
 ACT_KINDS = ("outlier", "channel_gain", "student_t3")
 
 
-def _gen(seed: int, stream: int) -> torch.Generator:
-    g = torch.Generator(device="cpu")
+def _gen(seed: int, stream: int, device: str = "cpu") -> torch.Generator:
+    g = torch.Generator(device=device)
     g.manual_seed(int(seed) * 1_000_003 + int(stream) * 7919 + 17)
     return g
 
 
-def activation(kind: str, M: int, K: int, seed: int, stream: int) -> torch.Tensor:
-    """BF16 [M, K] activation matrix drawn from the named distribution."""
-    g = _gen(seed, stream)
+def activation(kind: str, M: int, K: int, seed: int, stream: int,
+               device: str = "cpu") -> torch.Tensor:
+    """BF16 [M, K] activation matrix drawn from the named distribution.
+
+    device="cpu" is the reference stream used by the parity tests; another
+    device draws the same recipe from that device's generator (different
+    values, same distribution) -- used to build large benchmark inputs fast."""
+    g = _gen(seed, stream, device)
+    kw = dict(generator=g, dtype=torch.float32, device=device)
     if kind == "outlier":
-        x = torch.randn(M, K, generator=g, dtype=torch.float32)
-        mask = torch.rand(M, K, generator=g, dtype=torch.float32) < 0.01
+        x = torch.randn(M, K, **kw)
+        mask = torch.rand(M, K, **kw) < 0.01
         x = torch.where(mask, x * 20.0, x)
     elif kind == "channel_gain":
-        x = torch.randn(M, K, generator=g, dtype=torch.float32)
+        x = torch.randn(M, K, **kw)
         n_ch = int(round(0.02 * K))
-        ch = torch.randperm(K, generator=g)[:n_ch]
-        gain = torch.exp(torch.randn(n_ch, generator=g, dtype=torch.float32))
+        ch = torch.randperm(K, generator=g, device=device)[:n_ch]
+        gain = torch.exp(torch.randn(n_ch, **kw))
         x[:, ch] *= gain
     elif kind == "student_t3":
-        z = torch.randn(M, K, generator=g, dtype=torch.float32)
-        c = torch.randn(3, M, K, generator=g, dtype=torch.float32).pow_(2).sum(0)
+        z = torch.randn(M, K, **kw)
+        c = torch.randn(M, K, **kw).pow_(2)
+        c += torch.randn(M, K, **kw).pow_(2)
+        c += torch.randn(M, K, **kw).pow_(2)
         x = z / torch.sqrt(c / 3.0)
     else:
         raise ValueError(f"unknown activation kind {kind!r}")
     return x.to(torch.bfloat16)
 
 
-def weight(N: int, K: int, std: float, seed: int, stream: int) -> torch.Tensor:
+def weight(N: int, K: int, std: float, seed: int, stream: int,
+           device: str = "cpu") -> torch.Tensor:
     """BF16 [N, K] weight matrix ~ N(0, std)."""
-    g = _gen(seed, stream)
-    w = torch.randn(N, K, generator=g, dtype=torch.float32)
+    g = _gen(seed, stream, device)
+    w = torch.randn(N, K, generator=g, dtype=torch.float32, device=device)
     w.mul_(std)
     return w.to(torch.bfloat16)
 
@@ -90,7 +99,7 @@ WORKLOADS: Dict[str, Workload] = {
     "tiny": Workload("tiny linear 128x256x256", 128, "outlier", 0,
                      (Linear("w", 256, 256, 0.02),), (1,)),
     "llama3_8b_qkv_o": Workload(
-        "llama3-8b qkv+o prefill, 8192 tokens", 8192, "outlier", 1,
+        "llama3-8b qkv+o prefill, 8192 tokens", 8192, "channel_gain", 1,
         (Linear("qkv", 6144, 4096, 0.02), Linear("o", 4096, 4096, 0.02)), (1,)),
     "llama3_8b_mlp": Workload(
         "llama3-8b swiglu mlp prefill, 8192 tokens", 8192, "outlier", 2,
@@ -108,10 +117,11 @@ WORKLOADS: Dict[str, Workload] = {
 }
 
 
-def layer_weights(wl: Workload) -> List[torch.Tensor]:
+def layer_weights(wl: Workload, device: str = "cpu") -> List[torch.Tensor]:
     """All weights of a workload, stream ids 100 + position."""
-    return [weight(l.N, l.K, l.std, wl.seed, 100 + i) for i, l in enumerate(wl.linears)]
+    return [weight(l.N, l.K, l.std, wl.seed, 100 + i, device) for i, l in enumerate(wl.linears)]
 
 
-def layer_activation(wl: Workload, K: int, stream: int, M: int | None = None) -> torch.Tensor:
-    return activation(wl.act, wl.M if M is None else M, K, wl.seed, stream)
+def layer_activation(wl: Workload, K: int, stream: int, M: int | None = None,
+                     device: str = "cpu") -> torch.Tensor:
+    return activation(wl.act, wl.M if M is None else M, K, wl.seed, stream, device)
