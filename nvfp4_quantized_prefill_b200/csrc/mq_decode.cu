@@ -46,6 +46,8 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(const uint4 *__rest
                                                              unsigned *__restrict__ counters) {
     __shared__ float part[kWarps][128];
     __shared__ int last;
+    griddep_wait();
+    griddep_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t4 = lane & 3;
     const int group = blockIdx.x / S, slice = blockIdx.x - group * S;
@@ -145,11 +147,12 @@ cudaError_t launch_decode(const void *x, int64_t M, const void *w, int64_t N, in
     const int grid = static_cast<int>(groups * S);
     for (int64_t m0 = 0; m0 < M; m0 += 8) {
         const int mg = static_cast<int>(M - m0 < 8 ? M - m0 : 8);
-        decode_kernel<<<grid, kWarps * 32, 0, s>>>(
+        cudaError_t e = launch_pdl(
+            decode_kernel, dim3(grid), dim3(kWarps * 32), 0, s,
             static_cast<const uint4 *>(x) + m0 * (K / 8), mg, static_cast<const uint4 *>(w),
             static_cast<int>(N), static_cast<int>(K), S, static_cast<__nv_bfloat16 *>(y) + m0 * N,
             partials, counters);
-        cudaError_t e = cudaGetLastError();
+        if (e == cudaSuccess) e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -190,6 +190,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     cluster_sync();  // the peer's barriers exist before any cross-CTA signal
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // the set-up above overlaps the previous kernel's tail; operands and
+    // outputs are touched only after it has completed
+    griddep_wait();
+    griddep_launch_dependents();
     const int num_tiles = p.tiles_m * p.tiles_n;
     const int pair = static_cast<int>(blockIdx.x >> 1);
     const int npairs = static_cast<int>(gridDim.x >> 1);
@@ -590,16 +594,16 @@ cudaError_t launch_gemm_nvf4(const CUtensorMap &tmap_a, const CUtensorMap &tmap_
         e = cudaFuncSetAttribute(gemm_nvf4_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kSmemBytes);
         if (e != cudaSuccess) return e;
-        gemm_nvf4_kernel<true><<<grid, kThreads, kSmemBytes, s>>>(tmap_a, tmap_b, tmap_sfa, tmap_sfb,
-                                                                   tmap_y, p);
+        e = launch_pdl(gemm_nvf4_kernel<true>, dim3(grid), dim3(kThreads), kSmemBytes, s, tmap_a,
+                       tmap_b, tmap_sfa, tmap_sfb, tmap_y, p);
     } else {
         e = cudaFuncSetAttribute(gemm_nvf4_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kSmemBytes);
         if (e != cudaSuccess) return e;
-        gemm_nvf4_kernel<false><<<grid, kThreads, kSmemBytes, s>>>(tmap_a, tmap_b, tmap_sfa, tmap_sfb,
-                                                                    tmap_y, p);
+        e = launch_pdl(gemm_nvf4_kernel<false>, dim3(grid), dim3(kThreads), kSmemBytes, s, tmap_a,
+                       tmap_b, tmap_sfa, tmap_sfb, tmap_y, p);
     }
-    return cudaGetLastError();
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace mq

@@ -5,8 +5,45 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <utility>
 
 namespace mq {
+
+// ---- programmatic dependent launch -------------------------------------------
+//
+// Every kernel of this library is launched with programmatic stream
+// serialization: it may start while the previous kernel in the stream is
+// finishing (its prologue overlaps that kernel's tail), and it calls
+// griddep_wait() before its first access to global memory that an earlier
+// kernel may write or read.  griddep_wait() returns once the previous grid has
+// completed and its memory is visible; because every kernel waits before its
+// own accesses, the ordering carries down the whole stream.  Each kernel
+// also allows its successor to launch early (griddep_launch_dependents()).
+// Both are no-ops for a kernel launched without the attribute.
+#ifdef __CUDACC__
+__device__ __forceinline__ void griddep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+#endif
 
 // ---- activation / weight quantization (mq_quant.cu) ------------------------
 

@@ -11,7 +11,11 @@
 //   q  = E2M1_satfinite(fp32(x * f)), sign taken from x.
 //
 // Both kernels are HBM-streaming: 16-byte vector loads, coalesced across the
-// warp, grids sized in multiples of the SM count.
+// warp, grids sized in multiples of the SM count.  amax keeps 8 independent
+// 16-byte loads per thread in flight (HBM latency x bandwidth needs ~64 KB in
+// flight per SM); quantize runs one resident wave of CTAs and walks the matrix
+// from its end back to its start, so that it first reads the rows that amax
+// read last -- the ones most likely still in L2.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <cuda_fp16.h>
@@ -22,16 +26,50 @@ namespace mq {
 
 namespace {
 
+// Tuning constants (compile-time overridable for sweeps).
+#ifndef MQ_AMAX_UNROLL
+#define MQ_AMAX_UNROLL 4
+#endif
+#ifndef MQ_AMAX_BLOCKS_PER_SM
+#define MQ_AMAX_BLOCKS_PER_SM 8
+#endif
+#ifndef MQ_AMAX_NO_ALLOCATE
+#define MQ_AMAX_NO_ALLOCATE 0
+#endif
+#ifndef MQ_QUANT_UNROLL
+#define MQ_QUANT_UNROLL 2
+#endif
+#ifndef MQ_QUANT_BLOCKS_PER_SM
+#define MQ_QUANT_BLOCKS_PER_SM 6
+#endif
+
 constexpr int kThreads = 256;
-constexpr int kAmaxUnroll = 4;
+constexpr int kAmaxUnroll = MQ_AMAX_UNROLL;
+constexpr int kAmaxBlocksPerSm = MQ_AMAX_BLOCKS_PER_SM;
 
 __device__ __forceinline__ uint4 ldg_v4(const uint4 *p) { return __ldg(p); }
+
+// streaming read that does not allocate in L1 (each byte is read once)
+__device__ __forceinline__ uint4 ldg_v4_stream(const uint4 *p) {
+#if MQ_AMAX_NO_ALLOCATE
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+#else
+    return __ldg(p);
+#endif
+}
 
 // max of |bf16| over the 8 values of a 16-byte vector, as 16-bit magnitude bits
 // (non-negative bf16 values order like their bit patterns).
 __device__ __forceinline__ uint32_t absmax8_bits(uint4 v) {
-    const uint32_t m = 0x7FFF7FFFu;
-    uint32_t a = __vmaxu2(__vmaxu2(v.x & m, v.y & m), __vmaxu2(v.z & m, v.w & m));
+    uint32_t a, b;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(a) : "r"(v.x), "r"(v.y));
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(b) : "r"(v.z), "r"(v.w));
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(a) : "r"(a), "r"(b));
+    a &= 0x7FFF7FFFu;
     return max(a & 0xFFFFu, a >> 16);
 }
 
@@ -47,28 +85,35 @@ __device__ __forceinline__ float block_max(float v, float *red) {
     return r;
 }
 
-__global__ void __launch_bounds__(kThreads) amax_kernel(const uint4 *__restrict__ x, uint32_t M,
-                                                        uint32_t vpr, uint64_t ldv,
-                                                        float *__restrict__ partials) {
+// Grid-stride over the [M, vpr] matrix of 16-byte vectors (row stride ldv
+// vectors); each round issues kAmaxUnroll loads before reducing them.
+__global__ void __launch_bounds__(kThreads, kAmaxBlocksPerSm)
+    amax_kernel(const uint4 *__restrict__ x, uint32_t M, uint32_t vpr, uint64_t ldv,
+                float *__restrict__ partials) {
     __shared__ float red[kThreads / 32];
+    griddep_wait();
+    griddep_launch_dependents();
     const uint32_t total = M * vpr;
     const uint32_t stride = gridDim.x * kThreads;
-    uint32_t i = blockIdx.x * kThreads + threadIdx.x;
+    const bool dense = ldv == vpr;
     uint32_t mx = 0;
-    for (; i + (kAmaxUnroll - 1) * stride < total; i += kAmaxUnroll * stride) {
+    for (uint32_t i = blockIdx.x * kThreads + threadIdx.x; i < total; i += kAmaxUnroll * stride) {
         uint4 v[kAmaxUnroll];
 #pragma unroll
         for (int u = 0; u < kAmaxUnroll; ++u) {
-            uint32_t idx = i + u * stride;
-            uint32_t r = idx / vpr, c = idx - r * vpr;
-            v[u] = ldg_v4(x + r * ldv + c);
+            const uint32_t idx = i + u * stride;
+            v[u] = make_uint4(0, 0, 0, 0);
+            if (idx < total) {
+                uint64_t off = idx;
+                if (!dense) {
+                    const uint32_t r = idx / vpr;
+                    off = r * ldv + (idx - r * vpr);
+                }
+                v[u] = ldg_v4_stream(x + off);
+            }
         }
 #pragma unroll
         for (int u = 0; u < kAmaxUnroll; ++u) mx = max(mx, absmax8_bits(v[u]));
-    }
-    for (; i < total; i += stride) {
-        uint32_t r = i / vpr, c = i - r * vpr;
-        mx = max(mx, absmax8_bits(ldg_v4(x + r * ldv + c)));
     }
     float m = block_max(__uint_as_float(mx << 16), red);
     if (threadIdx.x == 0) partials[blockIdx.x] = m;
@@ -86,10 +131,8 @@ __device__ __forceinline__ uint64_t sf_word_offset(uint32_t r, uint32_t cq, uint
            ((r >> 5) & 3u) * 4u;
 }
 
-#ifndef MQ_QUANT_HW_SIGN
-#define MQ_QUANT_HW_SIGN 1
-#endif
-constexpr int kQuantUnroll = 2;
+constexpr int kQuantUnroll = MQ_QUANT_UNROLL;
+constexpr int kQuantBlocksPerSm = MQ_QUANT_BLOCKS_PER_SM;
 
 // fp32(a / 6) for a non-negative finite BF16 value a, in three operations:
 // q0 = RN(a * RN(1/6)), r = RN(a - 6 q0) (exact by FMA), q = RN(r * RN(1/6) + q0).
@@ -102,14 +145,45 @@ __device__ __forceinline__ float div6_bf16(float a) {
     return __fmaf_rn(r, inv6, q0);
 }
 
-// Two E2M1 codes (lo in bits 3:0, hi in bits 7:4) of x * f, round-to-nearest-even,
-// saturating at 6, sign from x (the conversion keeps the sign of a product
-// that rounds to zero).
-__device__ __forceinline__ uint32_t e2m1x2_signed(float lo, float hi) {
+// max(|a|, |b|) per BF16 half, sign bits = sign(a) ^ sign(b) (mask them off
+// to read the magnitudes).
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Eight BF16 values (two per word, element 2j in the low half of word j)
+// times f, each product rounded to FP32 (packed f32x2 multiplies) and then to
+// E2M1 (round-to-nearest-even, saturating at 6, the sign of x kept even when
+// the code is zero); returns the four code bytes, element 2j in the low
+// nibble of byte j.
+__device__ __forceinline__ uint32_t e2m1x8(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3,
+                                           float f) {
     uint32_t out;
-    asm("{\n\t.reg .b8 b;\n\tcvt.rn.satfinite.e2m1x2.f32 b, %2, %1;\n\tcvt.u32.u8 %0, b;\n\t}"
+    asm("{\n\t"
+        ".reg .b8 c0, c1, c2, c3;\n\t"
+        ".reg .b64 f2, x0, x1, x2, x3;\n\t"
+        ".reg .b32 l0, h0, l1, h1, l2, h2, l3, h3;\n\t"
+        "mov.b64 f2, {%5, %5};\n\t"
+        "shl.b32 l0, %1, 16;\n\tand.b32 h0, %1, 0xFFFF0000;\n\t"
+        "shl.b32 l1, %2, 16;\n\tand.b32 h1, %2, 0xFFFF0000;\n\t"
+        "shl.b32 l2, %3, 16;\n\tand.b32 h2, %3, 0xFFFF0000;\n\t"
+        "shl.b32 l3, %4, 16;\n\tand.b32 h3, %4, 0xFFFF0000;\n\t"
+        "mov.b64 x0, {l0, h0};\n\tmov.b64 x1, {l1, h1};\n\t"
+        "mov.b64 x2, {l2, h2};\n\tmov.b64 x3, {l3, h3};\n\t"
+        "mul.rn.f32x2 x0, x0, f2;\n\tmul.rn.f32x2 x1, x1, f2;\n\t"
+        "mul.rn.f32x2 x2, x2, f2;\n\tmul.rn.f32x2 x3, x3, f2;\n\t"
+        "mov.b64 {l0, h0}, x0;\n\tmov.b64 {l1, h1}, x1;\n\t"
+        "mov.b64 {l2, h2}, x2;\n\tmov.b64 {l3, h3}, x3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 c0, h0, l0;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 c1, h1, l1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 c2, h2, l2;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 c3, h3, l3;\n\t"
+        "mov.b32 %0, {c0, c1, c2, c3};\n\t"
+        "}"
         : "=r"(out)
-        : "f"(lo), "f"(hi));
+        : "r"(w0), "r"(w1), "r"(w2), "r"(w3), "f"(f));
     return out;
 }
 
@@ -120,41 +194,32 @@ __device__ __forceinline__ uint32_t e2m1x2_signed(float lo, float hi) {
 __device__ __forceinline__ void quantize_block16(const uint32_t (&w)[8], float s_enc,
                                                  const float *ftab, uint32_t &lo, uint32_t &hi,
                                                  uint32_t &sb_out) {
-    const uint32_t m = 0x7FFF7FFFu;
-    uint32_t a = __vmaxu2(__vmaxu2(w[0] & m, w[1] & m), __vmaxu2(w[2] & m, w[3] & m));
-    a = __vmaxu2(a, __vmaxu2(__vmaxu2(w[4] & m, w[5] & m), __vmaxu2(w[6] & m, w[7] & m)));
+    uint32_t a = absmax_bf16x2(absmax_bf16x2(absmax_bf16x2(w[0], w[1]), absmax_bf16x2(w[2], w[3])),
+                               absmax_bf16x2(absmax_bf16x2(w[4], w[5]), absmax_bf16x2(w[6], w[7])));
+    a &= 0x7FFF7FFFu;
     const float amax_b = __uint_as_float(max(a & 0xFFFFu, a >> 16) << 16);
     const float sbf = __fmul_rn(div6_bf16(amax_b), s_enc);
     const uint32_t sb = __nv_cvt_float_to_fp8(sbf, __NV_SATFINITE, __NV_E4M3);
     const float f = ftab[sb];  // = dec(sb) == 0 ? 0 : fp32(s_enc / dec(sb))
-    uint32_t byte[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const float x0 = __uint_as_float(w[j] << 16);
-        const float x1 = __uint_as_float(w[j] & 0xFFFF0000u);
-#if MQ_QUANT_HW_SIGN
-        byte[j] = e2m1x2_signed(__fmul_rn(x0, f), __fmul_rn(x1, f));
-#else
-        byte[j] = e2m1x2_signed(fabsf(__fmul_rn(x0, f)), fabsf(__fmul_rn(x1, f))) |
-                  ((w[j] >> 12) & 0x8u) | ((w[j] >> 24) & 0x80u);
-#endif
-    }
-    lo = byte[0] | (byte[1] << 8) | (byte[2] << 16) | (byte[3] << 24);
-    hi = byte[4] | (byte[5] << 8) | (byte[6] << 16) | (byte[7] << 24);
+    lo = e2m1x8(w[0], w[1], w[2], w[3], f);
+    hi = e2m1x8(w[4], w[5], w[6], w[7], f);
     sb_out = sb;
 }
 
 // Each warp quantizes 512-element row segments (lane l: 16-block l of the
 // segment, two 16-byte loads), kQuantUnroll segments per iteration with all
-// loads issued first.  Lanes 4t..4t+3 hold the 4 scales of one swizzled
-// 32-bit scale word.
-__global__ void __launch_bounds__(kThreads) quantize_kernel(
+// loads issued first; segments are taken from the last one backwards.  Lanes
+// 4t..4t+3 hold the 4 scales of one swizzled 32-bit scale word.
+__global__ void __launch_bounds__(kThreads, kQuantBlocksPerSm) quantize_kernel(
     const uint4 *__restrict__ x, uint32_t M, uint32_t K, uint64_t ldv,
     const float *__restrict__ partials, int n_partials, uint2 *__restrict__ codes,
     uint8_t *__restrict__ sf, float *__restrict__ s_enc_out, uint32_t Mpad) {
     __shared__ float red[kThreads / 32];
     __shared__ float ftab[128];
+    griddep_wait();
+    griddep_launch_dependents();
     float amx = 0.0f;
+#pragma unroll 4
     for (int i = threadIdx.x; i < n_partials; i += kThreads) amx = fmaxf(amx, partials[i]);
     const float amax = block_max(amx, red);
     float s_enc = __fdiv_rn(2688.0f, amax);
@@ -173,25 +238,43 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t nwarps = gridDim.x * (kThreads / 32);
     const uint32_t warp_id = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    // Segment seg = total - 1 - pos for pos = warp_id, warp_id + nwarps, ...;
+    // (row, segment-in-row) of the current seg is stepped back by nwarps
+    // segments at a time: dq rows and dr segments.
+    const uint32_t dq = nwarps / segs, dr = nwarps - (nwarps / segs) * segs;
+    uint32_t r0 = 0, s0 = 0;
+    if (warp_id < total) {
+        const uint32_t seg = total - 1u - warp_id;
+        r0 = seg / segs;
+        s0 = seg - r0 * segs;
+    }
+    auto step_back = [&](uint32_t &r, uint32_t &sg) {
+        if (sg >= dr) {
+            sg -= dr;
+            r -= dq;
+        } else {
+            sg += segs - dr;
+            r -= dq + 1u;
+        }
+    };
     for (uint32_t base = warp_id; base < total; base += nwarps * kQuantUnroll) {
         uint32_t w[kQuantUnroll][8];
         uint32_t rr[kQuantUnroll], bb[kQuantUnroll];
         bool act[kQuantUnroll];
 #pragma unroll
         for (int u = 0; u < kQuantUnroll; ++u) {
-            const uint32_t seg = base + u * nwarps;
-            const uint32_t r = seg / segs, sg = seg - r * segs;
-            rr[u] = r;
-            bb[u] = sg * 32u + lane;  // block index within the row
-            act[u] = seg < total && bb[u] < kblocks;
+            rr[u] = r0;
+            bb[u] = s0 * 32u + lane;  // block index within the row
+            act[u] = base + u * nwarps < total && bb[u] < kblocks;
             uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
             if (act[u]) {
-                const uint4 *px = x + r * ldv + bb[u] * 2u;
+                const uint4 *px = x + r0 * ldv + bb[u] * 2u;
                 v0 = ldg_v4(px);
                 v1 = ldg_v4(px + 1);
             }
             w[u][0] = v0.x; w[u][1] = v0.y; w[u][2] = v0.z; w[u][3] = v0.w;
             w[u][4] = v1.x; w[u][5] = v1.y; w[u][6] = v1.z; w[u][7] = v1.w;
+            step_back(r0, s0);
         }
 #pragma unroll
         for (int u = 0; u < kQuantUnroll; ++u) {
@@ -222,7 +305,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(
 int amax_grid(int64_t M, int64_t K, int num_sms) {
     const int64_t vecs = M * (K / 8);
     int64_t g = (vecs + kThreads * kAmaxUnroll - 1) / (kThreads * kAmaxUnroll);
-    const int64_t cap = 4LL * num_sms;
+    const int64_t cap = static_cast<int64_t>(kAmaxBlocksPerSm) * num_sms;
     if (g > cap) g = cap;
     if (g < 1) g = 1;
     return static_cast<int>(g);
@@ -230,27 +313,35 @@ int amax_grid(int64_t M, int64_t K, int num_sms) {
 
 cudaError_t launch_amax(const void *x, int64_t M, int64_t K, int64_t ldx, float *partials,
                         int grid, cudaStream_t s) {
-    amax_kernel<<<grid, kThreads, 0, s>>>(static_cast<const uint4 *>(x),
-                                          static_cast<uint32_t>(M),
-                                          static_cast<uint32_t>(K / 8),
-                                          static_cast<uint64_t>(ldx / 8), partials);
-    return cudaGetLastError();
+    return launch_pdl(amax_kernel, dim3(grid), dim3(kThreads), 0, s, static_cast<const uint4 *>(x),
+                      static_cast<uint32_t>(M), static_cast<uint32_t>(K / 8),
+                      static_cast<uint64_t>(ldx / 8), partials);
 }
 
 cudaError_t launch_quantize(const void *x, int64_t M, int64_t K, int64_t ldx,
                             const float *partials, int n_partials, uint8_t *codes,
                             uint8_t *sf_swizzled, float *s_enc, int num_sms, cudaStream_t s) {
+    // one resident wave: every CTA pays the scale-table prologue once
+    static int resident = 0;
+    if (resident == 0) {
+        int b = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, quantize_kernel, kThreads, 0) !=
+                cudaSuccess ||
+            b < 1)
+            b = 1;
+        resident = b;
+    }
     const int64_t segs = M * ((K + 511) / 512);
     int64_t g = (segs + (kThreads / 32) - 1) / (kThreads / 32);
-    const int64_t cap = 8LL * num_sms;
+    const int64_t cap = static_cast<int64_t>(resident) * num_sms;
     if (g > cap) g = cap;
     if (g < 1) g = 1;
     const int64_t Mpad = (M + 127) / 128 * 128;
-    quantize_kernel<<<static_cast<int>(g), kThreads, 0, s>>>(
-        static_cast<const uint4 *>(x), static_cast<uint32_t>(M), static_cast<uint32_t>(K),
-        static_cast<uint64_t>(ldx / 8), partials, n_partials, reinterpret_cast<uint2 *>(codes),
-        sf_swizzled, s_enc, static_cast<uint32_t>(Mpad));
-    return cudaGetLastError();
+    return launch_pdl(quantize_kernel, dim3(static_cast<unsigned>(g)), dim3(kThreads), 0, s,
+                      static_cast<const uint4 *>(x), static_cast<uint32_t>(M),
+                      static_cast<uint32_t>(K), static_cast<uint64_t>(ldx / 8), partials,
+                      n_partials, reinterpret_cast<uint2 *>(codes), sf_swizzled, s_enc,
+                      static_cast<uint32_t>(Mpad));
 }
 
 }  // namespace mq
