@@ -15,15 +15,26 @@
 //                tiles and both B scale halves, into a 5-stage ring; every
 //                load completes on the even CTA's stage barriers (scale tiles
 //                on their own, so their TMEM copies overlap the operand loads).
-//   warp 1       (even CTA) MMA issuer: 4 paired MMAs (K = 64 each) per stage
-//                into a 128 x 256 FP32 accumulator in each CTA's TMEM.
+//   warp 1       (even CTA) MMA issuer: one wait per stage, then 4 paired
+//                MMAs (K = 64 each) and the stage's commit from one issue
+//                block, into a 128 x 256 FP32 accumulator in each CTA's TMEM.
 //   warps 2-3    (even CTA) scale copiers: tcgen05.cp of the stage's scale
-//                tiles into both CTAs' TMEM, from their own threads -- a
-//                thread's tcgen05 instructions run in order, so copies issued
-//                by the MMA thread would queue ahead of its MMAs.
+//                tiles into both CTAs' TMEM (6 copies per copier per stage in
+//                one issue block), from their own threads -- a thread's
+//                tcgen05 instructions run in order, so copies issued by the
+//                MMA thread would queue ahead of its MMAs; a copier commits
+//                the stage's sf_full only after the operand barrier too.
+//                Each tcgen05 instruction, barrier wait and commit costs the
+//                issuing warp ~80-100 cycles, against ~550 cycles of tensor
+//                work per stage: the issue paths are trimmed to stay below.
 //   warps 4-11   (both CTAs) epilogue: drain the CTA's accumulator half with
-//                tcgen05.ld, release it to the MMA thread, then scale, round to
-//                BF16 and store while the next tile's main loop runs.
+//                tcgen05.ld, meet on a named barrier, and release it with one
+//                arrive per CTA (CTA-scope release: the cluster-scope form
+//                stalls the arriving thread for ~0.7 us, all of it on the
+//                tensor pipe's idle time between tiles); then store while the
+//                next tile's main loop runs.  The SwiGLU variant computes
+//                SiLU(gate) * up only after the release.  Warpgroup 0 hands
+//                registers to the epilogue warpgroups (setmaxnreg).
 // Every mbarrier wait is bounded (about two seconds); on a timeout the kernel
 // latches an error bit, stops issuing work, lets issued copies and MMAs land,
 // frees its tensor memory and exits.
@@ -44,9 +55,8 @@ namespace {
 #ifndef MQ_GEMM_GROUP_M
 #define MQ_GEMM_GROUP_M 8
 #endif
-#ifndef MQ_GEMM_COPIERS
-#define MQ_GEMM_COPIERS 2
-#endif
+
+
 
 constexpr int kStages = MQ_GEMM_STAGES;
 constexpr uint32_t kABytes = 128 * 128;          // this CTA's 128 A rows x 128 B (256 fp4)
@@ -60,7 +70,7 @@ constexpr uint32_t kStageTileBytes = 32 * 128;    // epilogue staging: 32 rows x
 constexpr uint32_t kStagingBytes = 8 * kStageTileBytes;  // one per epilogue warp
 constexpr uint32_t kBarBytes = 256;
 constexpr uint32_t kSmemBytes = kStages * kStageBytes + kStagingBytes + kBarBytes + 1024;
-constexpr int kCopiers = MQ_GEMM_COPIERS;        // scale-copy warps (0: the MMA thread copies)
+constexpr int kCopiers = 2;                      // scale-copy warps
 constexpr int kEpiWarp0 = 2 + kCopiers;          // first of 8 epilogue warps
 constexpr int kThreads = 32 * (kEpiWarp0 + 8);
 constexpr uint32_t kTmemCols = 512;
@@ -69,6 +79,12 @@ constexpr uint32_t kSfColsPerStage = 48;         // 16 for A + 32 for B
 constexpr int kGroupM = MQ_GEMM_GROUP_M;         // tile raster: M-tiles per group
 constexpr uint16_t kPairMask = 0x3;
 
+constexpr int kRegsLaunch = 168;                 // per thread, from __launch_bounds__(kThreads, 1)
+constexpr int kRegsLow = 56;                     // warpgroup 0 after setmaxnreg.dec
+constexpr int kRegsHigh = 224;                   // epilogue warpgroups after setmaxnreg.inc
+static_assert(kEpiWarp0 == 4, "warpgroup 0 = producer, MMA, copiers; 1-2 = epilogue");
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsLaunch, "register split");
+static_assert(kThreads * kRegsLaunch <= 65536, "launch register file");
 static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
 static_assert(kSfCol + kStages * kSfColsPerStage <= kTmemCols, "TMEM budget");
 static_assert((4 * kStages + 4) * 8 + 48 <= kBarBytes, "barrier area");
@@ -169,13 +185,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int s = 0; s < kStages; ++s) {
             mbar_init(bar0 + 8u * s, 1);             // arrive.expect_tx of the even CTA
             mbar_init(empty0 + 8u * s, 1);           // MMA commit (to both CTAs)
-            mbar_init(sf_full0 + 8u * s, kCopiers > 0 ? kCopiers : 1);  // one commit per copier
+            mbar_init(sf_full0 + 8u * s, kCopiers);  // one commit per copier
             mbar_init(sfd_full0 + 8u * s, 1);        // arrive.expect_tx of the even CTA
         }
         mbar_init(acc_full, 1);
-        mbar_init(acc_empty, 16);                    // 8 epilogue warps x 2 CTAs
+        mbar_init(acc_empty, 2);                     // one arrive per CTA's epilogue
         mbar_init(drain_bar, 1);
-        mbar_init(sf_drain_bar, kCopiers > 0 ? kCopiers : 1);
+        mbar_init(sf_drain_bar, kCopiers);
         *abort_flag = 0;
         fence_barrier_init();
         prefetch_tmap(&tmap_a);
@@ -201,6 +217,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // The producer, MMA and copier roles run their loops on all 32 lanes with
     // warp-uniform state; one elected lane issues each TMA / tcgen05
     // instruction (see the warp_* wrappers).
+    // Registers: warpgroup 0 (producer, MMA, copiers) gives most of its share
+    // to the two epilogue warpgroups, which hold a whole 128-column
+    // accumulator row slice: 128 x 56 + 256 x 224 = 384 x 168 (the launch).
+    if (warp < kEpiWarp0) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         int stage = 0;
@@ -273,10 +294,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 if (!warp_mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag, p.err)) break;
                 tc_fence_after();
                 for (int kt = 0; kt < p.k_tiles; ++kt) {
-                    // the stage's scales are in TMEM and both CTAs' operands landed
-                    const uint32_t sf_bar = kCopiers > 0 ? sf_full0 : sfd_full0;
-                    if (!warp_mbar_wait(sf_bar + 8u * stage, phase, abort_flag, p.err) ||
-                        !warp_mbar_wait(bar0 + 8u * stage, phase, abort_flag, p.err)) {
+                    // the stage's scales are in TMEM and both CTAs' operands
+                    // landed: the copiers commit sf_full only after seeing the
+                    // operand barrier, so this is the one wait per stage
+                    if (!warp_mbar_wait(sf_full0 + 8u * stage, phase, abort_flag, p.err)) {
                         ok = false;
                         break;
                     }
@@ -286,23 +307,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const uint32_t sB = sA + kABytes;
                     const uint32_t tsfa = tmem + kSfCol + stage * kSfColsPerStage;
                     const uint32_t tsfb = tsfa + 16u;
-                    if (kCopiers == 0) {
-                        // in-thread copies: ordered before this thread's MMAs below
-                        const uint32_t sSFA = sB + kBBytes;
-                        const uint32_t sSFB = sSFA + kSfaBytes;
-                        for (int a = 0; a < natoms; ++a) {
-                            warp_cp_sf_pair(tsfa + 4u * a, sdesc_sf_tile(sSFA + 512u * a));
-                            warp_cp_sf_pair(tsfb + 8u * a, sdesc_sf_tile(sSFB + 512u * a));
-                            warp_cp_sf_pair(tsfb + 8u * a + 4u,
-                                            sdesc_sf_tile(sSFB + 4u * 512u + 512u * a));
+                    if (natoms == 4) {
+                        warp_mma4_commit_pair(tmem, sdesc_kmajor_sw128(sA), sdesc_kmajor_sw128(sB), idesc,
+                                              tsfa, tsfb, kt != 0 ? 1u : 0u, empty0 + 8u * stage,
+                                              kPairMask);
+                    } else {
+                        for (int kb = 0; kb < natoms; ++kb) {
+                            warp_mma_nvf4_pair(tmem, sdesc_kmajor_sw128(sA + 32u * kb),
+                                               sdesc_kmajor_sw128(sB + 32u * kb), idesc, tsfa + 4u * kb,
+                                               tsfb + 8u * kb, (kt | kb) != 0 ? 1u : 0u);
                         }
+                        warp_commit_pair_mc(empty0 + 8u * stage, kPairMask);  // frees both CTAs' stage
                     }
-                    for (int kb = 0; kb < natoms; ++kb) {
-                        warp_mma_nvf4_pair(tmem, sdesc_kmajor_sw128(sA + 32u * kb),
-                                           sdesc_kmajor_sw128(sB + 32u * kb), idesc, tsfa + 4u * kb,
-                                           tsfb + 8u * kb, (kt | kb) != 0 ? 1u : 0u);
-                    }
-                    warp_commit_pair_mc(empty0 + 8u * stage, kPairMask);  // frees both CTAs' stage
                     if (++stage == kStages) {
                         stage = 0;
                         phase ^= 1u;
@@ -316,7 +332,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             warp_commit_pair(drain_bar);
             drain_wait(drain_bar, 0, p.err);
         }
-    } else if (warp < kEpiWarp0) {
+    } else {
         // ------------------------------------------------------------ scale copiers
         // Copier c copies k-blocks c, c + kCopiers, ... of each stage: the A
         // scale tile (each CTA its own rows) and both B halves, into the
@@ -338,10 +354,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const uint32_t sSFB = sSFA + kSfaBytes;
                     const uint32_t tsfa = tmem + kSfCol + stage * kSfColsPerStage;
                     const uint32_t tsfb = tsfa + 16u;
-                    for (int a = cid; a < natoms; a += kCopiers) {
-                        warp_cp_sf_pair(tsfa + 4u * a, sdesc_sf_tile(sSFA + 512u * a));
-                        warp_cp_sf_pair(tsfb + 8u * a, sdesc_sf_tile(sSFB + 512u * a));
-                        warp_cp_sf_pair(tsfb + 8u * a + 4u, sdesc_sf_tile(sSFB + 4u * 512u + 512u * a));
+                    if (natoms == 4) {
+                        const uint32_t a = static_cast<uint32_t>(cid);
+                        warp_cp6_pair(tsfa + 4u * a, tsfb + 8u * a, sdesc_sf_tile(sSFA + 512u * a),
+                                      sdesc_sf_tile(sSFB + 512u * a),
+                                      sdesc_sf_tile(sSFB + 4u * 512u + 512u * a));
+                    } else {
+                        for (int a = cid; a < natoms; a += kCopiers) {
+                            warp_cp_sf_pair(tsfa + 4u * a, sdesc_sf_tile(sSFA + 512u * a));
+                            warp_cp_sf_pair(tsfb + 8u * a, sdesc_sf_tile(sSFB + 512u * a));
+                            warp_cp_sf_pair(tsfb + 8u * a + 4u,
+                                            sdesc_sf_tile(sSFB + 4u * 512u + 512u * a));
+                        }
+                    }
+                    // the operands too have landed when sf_full completes, so
+                    // the MMA thread waits on one barrier per stage
+                    if (!warp_mbar_wait(bar0 + 8u * stage, phase, abort_flag, p.err)) {
+                        ok = false;
+                        break;
                     }
                     warp_commit_pair(sf_full0 + 8u * stage);
                     if (++stage == kStages) {
@@ -353,7 +383,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             warp_commit_pair(sf_drain_bar);
             drain_wait(sf_drain_bar, 0, p.err);
         }
+    }
     } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
         // ------------------------------------------------------------ epilogue
         const int ew = warp - kEpiWarp0;  // 0..7
         const int sub = warp & 3;         // TMEM lane group this warp may read
@@ -361,6 +393,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const float alpha = __frcp_rn(__fmul_rn(*p.s_enc_a, *p.s_enc_b));
         const bool vec_ok = (p.ldy % 8) == 0;
         const uint32_t acc_empty_pair = mapa_shared(acc_empty, 0);
+        // The accumulator may be overwritten once all 8 epilogue warps of both
+        // CTAs have their tcgen05.ld data in registers: the warps meet on a
+        // named barrier and one thread per CTA arrives on the MMA thread's
+        // acc_empty (count 2).
+        // `got`: this warp saw the accumulator complete (false after an
+        // abort); the barrier's AND keeps the 8 warps leaving together.
+        auto release_acc = [&](bool got) -> bool {
+            tc_fence_before();
+            uint32_t all;
+            asm volatile(
+                "{\n\t.reg .pred p, q;\n\t"
+                "setp.ne.u32 p, %1, 0;\n\t"
+                "bar.red.and.pred q, 2, 256, p;\n\t"
+                "selp.u32 %0, 1, 0, q;\n\t}"
+                : "=r"(all)
+                : "r"(got ? 1u : 0u)
+                : "memory");
+            if (!all) return false;
+            if (ew == 0 && lane == 0) {
+                if (rank == 0)
+                    mbar_arrive(acc_empty);
+                else
+                    mbar_arrive_remote(acc_empty_pair);
+            }
+            return true;
+        };
         // this warp's staging tile: 32 rows of 128 bytes, 128-byte swizzled
         // (16-byte chunk j of row r at r * 128 + ((j ^ (r % 8)) * 16)), the
         // layout the output tensor map's SWIZZLE_128B store reads
@@ -388,31 +446,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int tm, tn;
             tile_coords(t, p.tiles_m, p.tiles_n, tm, tn);
             // warp-uniform decision: the TMEM loads below are .sync.aligned
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait(acc_full, acc_phase, abort_flag, p.err))) break;
-            tc_fence_after();
+            const bool got = __all_sync(0xFFFFFFFFu, mbar_wait(acc_full, acc_phase, abort_flag, p.err));
+            if (got) tc_fence_after();
             const int row0 = tm * 256 + static_cast<int>(rank) * 128 + sub * 32;
             const int row = row0 + lane;
             const uint32_t tbase = tmem + (static_cast<uint32_t>(sub * 32) << 16);
             if (!kSwiglu) {
+                // two rounds of 64 columns: load, scale and round; then release
+                // (measured faster than loading all 128 before the release)
                 uint32_t packed[64];
+                if (got) {
 #pragma unroll
-                for (int c = 0; c < 4; c += 2) {
-                    uint32_t r0[32], r1[32];
-                    tmem_ld32(tbase + half * 128 + c * 32, r0);
-                    tmem_ld32(tbase + half * 128 + (c + 1) * 32, r1);
-                    tmem_ld_wait();
+                    for (int c = 0; c < 4; c += 2) {
+                        uint32_t r0[32], r1[32];
+                        tmem_ld32(tbase + half * 128 + c * 32, r0);
+                        tmem_ld32(tbase + half * 128 + (c + 1) * 32, r1);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        packed[c * 16 + j] = pack_bf16x2(__fmul_rn(alpha, __uint_as_float(r0[2 * j])),
-                                                         __fmul_rn(alpha, __uint_as_float(r0[2 * j + 1])));
-                        packed[(c + 1) * 16 + j] =
-                            pack_bf16x2(__fmul_rn(alpha, __uint_as_float(r1[2 * j])),
-                                        __fmul_rn(alpha, __uint_as_float(r1[2 * j + 1])));
+                        for (int j = 0; j < 16; ++j) {
+                            packed[c * 16 + j] = pack_bf16x2(__fmul_rn(alpha, __uint_as_float(r0[2 * j])),
+                                                             __fmul_rn(alpha, __uint_as_float(r0[2 * j + 1])));
+                            packed[(c + 1) * 16 + j] =
+                                pack_bf16x2(__fmul_rn(alpha, __uint_as_float(r1[2 * j])),
+                                            __fmul_rn(alpha, __uint_as_float(r1[2 * j + 1])));
+                        }
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(acc_empty_pair);
+                if (!release_acc(got)) break;
                 const int n0 = tn * 256 + half * 128;
                 if (p.tma_store) {
                     if (row0 < p.M && n0 < p.N) {
@@ -424,29 +484,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                    vec_ok);
                 }
             } else {
+                // gate columns [64 half, +64) and the matching up columns
+                // (128 + ...) into registers, release, then SwiGLU
+                uint32_t rg[2][32], ru[2][32];
+                if (got) {
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        tmem_ld32(tbase + half * 64 + c * 32, rg[c]);
+                        tmem_ld32(tbase + 128 + half * 64 + c * 32, ru[c]);
+                    }
+                    tmem_ld_wait();
+                }
+                if (!release_acc(got)) break;
                 uint32_t packed[32];
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
-                    uint32_t rg[32], ru[32];
-                    tmem_ld32(tbase + half * 64 + c * 32, rg);
-                    tmem_ld32(tbase + 128 + half * 64 + c * 32, ru);
-                    tmem_ld_wait();
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         float hv[2];
 #pragma unroll
                         for (int e = 0; e < 2; ++e) {
-                            const float g = bf16_round(__fmul_rn(alpha, __uint_as_float(rg[2 * j + e])));
-                            const float u = bf16_round(__fmul_rn(alpha, __uint_as_float(ru[2 * j + e])));
+                            const float g = bf16_round(__fmul_rn(alpha, __uint_as_float(rg[c][2 * j + e])));
+                            const float u = bf16_round(__fmul_rn(alpha, __uint_as_float(ru[c][2 * j + e])));
                             const float silu = __fdiv_rn(g, __fadd_rn(1.0f, expf(-g)));
                             hv[e] = __fmul_rn(silu, u);
                         }
                         packed[c * 16 + j] = pack_bf16x2(hv[0], hv[1]);
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(acc_empty_pair);
                 const int n0 = tn * 128 + half * 64;
                 if (row < p.M) {
 #pragma unroll

@@ -155,6 +155,15 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
 }
 
 // Arrive on an mbarrier given by a shared::cluster address (any CTA of the cluster).
+// Arrive on a barrier of the peer CTA with release semantics at CTA scope:
+// the signal carries no data the waiter reads through memory, and the
+// cluster-scope release form stalls the arriving thread for several hundred
+// nanoseconds.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                  : "memory");
@@ -267,6 +276,64 @@ __device__ __forceinline__ void warp_mma_nvf4_pair(uint32_t d_tmem, uint64_t ade
         "@e tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16"
         " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+// One K = 256 stage: four paired MMAs (K = 64 each; the A / B descriptors
+// advance 32 bytes = 2 descriptor units, the scale columns by 4 / 8) and the
+// commit that frees the stage in both CTAs, from one elected lane.  The first
+// MMA overwrites the accumulator when `accumulate` is 0.
+__device__ __forceinline__ void warp_mma4_commit_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                      uint32_t idesc, uint32_t sfa_tmem,
+                                                      uint32_t sfb_tmem, uint32_t accumulate,
+                                                      uint32_t bar, uint16_t cta_mask) {
+    asm volatile(
+        "{\n\t.reg .pred p, t, e;\n\t"
+        ".reg .b64 a1, a2, a3, b1, b2, b3;\n\t"
+        ".reg .b32 sa1, sa2, sa3, sb1, sb2, sb3;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.b32 t, 0, 0;\n\t"
+        "add.s64 a1, %1, 2;\n\tadd.s64 a2, %1, 4;\n\tadd.s64 a3, %1, 6;\n\t"
+        "add.s64 b1, %2, 2;\n\tadd.s64 b2, %2, 4;\n\tadd.s64 b3, %2, 6;\n\t"
+        "add.u32 sa1, %5, 4;\n\tadd.u32 sa2, %5, 8;\n\tadd.u32 sa3, %5, 12;\n\t"
+        "add.u32 sb1, %6, 8;\n\tadd.u32 sb2, %6, 16;\n\tadd.u32 sb3, %6, 24;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16"
+        " [%0], %1, %2, %3, [%5], [%6], p;\n\t"
+        "@e tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16"
+        " [%0], a1, b1, %3, [sa1], [sb1], t;\n\t"
+        "@e tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16"
+        " [%0], a2, b2, %3, [sa2], [sb2], t;\n\t"
+        "@e tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16"
+        " [%0], a3, b3, %3, [sa3], [sb3], t;\n\t"
+        "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%7], %8;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem),
+        "r"(bar), "h"(cta_mask)
+        : "memory");
+}
+
+// A copier's share of one stage when two copiers split its four K-blocks:
+// K-blocks kb and kb + 2, each its A scale tile and the two B scale tiles
+// (512-byte tiles; kb + 2 is 1024 bytes = 64 descriptor units further, and
+// 8 / 16 TMEM columns further), from one elected lane.
+__device__ __forceinline__ void warp_cp6_pair(uint32_t tsfa, uint32_t tsfb, uint64_t da,
+                                              uint64_t db_lo, uint64_t db_hi) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        ".reg .b64 a2, l2, h2;\n\t"
+        ".reg .b32 ta2, tb1, tb2, tb3;\n\t"
+        "add.s64 a2, %2, 64;\n\tadd.s64 l2, %3, 64;\n\tadd.s64 h2, %4, 64;\n\t"
+        "add.u32 ta2, %0, 8;\n\tadd.u32 tb1, %1, 4;\n\t"
+        "add.u32 tb2, %1, 16;\n\tadd.u32 tb3, %1, 20;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %2;\n\t"
+        "@e tcgen05.cp.cta_group::2.32x128b.warpx4 [%1], %3;\n\t"
+        "@e tcgen05.cp.cta_group::2.32x128b.warpx4 [tb1], %4;\n\t"
+        "@e tcgen05.cp.cta_group::2.32x128b.warpx4 [ta2], a2;\n\t"
+        "@e tcgen05.cp.cta_group::2.32x128b.warpx4 [tb2], l2;\n\t"
+        "@e tcgen05.cp.cta_group::2.32x128b.warpx4 [tb3], h2;\n\t}"
+        ::"r"(tsfa), "r"(tsfb), "l"(da), "l"(db_lo), "l"(db_hi)
         : "memory");
 }
 
