@@ -223,29 +223,51 @@ class Prefill:
         self.ops = []    # list of (name, callable) kernel launches, in order
         self.flops = 0.0
         if wl.swiglu:
-            # pairs of (gate_up, down)
+            # gate_up followed by down is one SwiGLU MLP (the GEMM epilogue
+            # writes h and its amax); every other projection is a plain linear
+            # with its own activation
             self.xs = []
-            for i in range(0, len(self.W), 2):
-                Wgu, Wd = self.W[i], self.W[i + 1]
-                I = Wgu.N // 2
-                x = workloads.layer_activation(wl, Wgu.K, i, device=str(dev))
-                self.xs.append(x)
-                qx, qh = qbuf(Wgu.K), qbuf(I)
-                h = torch.empty(M, I, dtype=bf, device=dev)
-                y = torch.empty(M, Wd.N, dtype=bf, device=dev)
-                self._add_quant(f"amax+quant x{i}", x, Wgu.K, qx)
-                self.ops.append((f"gemm {wl.linears[i].name}+swiglu", "gemm",
-                                 lambda st, qx=qx, Wgu=Wgu, h=h, qh=qh: qh.__setitem__(
-                                     "n", mq.mq_gemm_nvfp4_swiglu(qx["codes"], qx["sf"], qx["s"], M,
-                                                                  Wgu.handle, h, qh["part"], st))))
-                self.ops.append((f"quant h{i}", "quant",
-                                 lambda st, h=h, qh=qh, I=I: mq.mq_quantize_nvfp4(
-                                     h, M, I, I, qh["codes"], qh["sf"], qh["s"],
-                                     amax_partials=qh["part"], n_partials=qh["n"], stream=st)))
-                self.ops.append((f"gemm {wl.linears[i + 1].name}", "gemm",
-                                 lambda st, qh=qh, Wd=Wd, y=y: mq.mq_gemm_nvfp4(
-                                     qh["codes"], qh["sf"], qh["s"], M, Wd.handle, y, Wd.N, st)))
-                self.flops += 2.0 * M * Wgu.N * Wgu.K + 2.0 * M * Wd.N * Wd.K
+            self.plan = []   # ("mlp", gate_up index, down index, x index) / ("linear", index, x index)
+            lin = list(wl.linears)
+            i = 0
+            while i < len(lin):
+                W = self.W[i]
+                if lin[i].name == "gate_up" and i + 1 < len(lin) and lin[i + 1].name == "down":
+                    Wgu, Wd = self.W[i], self.W[i + 1]
+                    I = Wgu.N // 2
+                    assert Wd.K == I, "down projection K must equal the SwiGLU width"
+                    x = workloads.layer_activation(wl, Wgu.K, i, device=str(dev))
+                    self.plan.append(("mlp", i, i + 1, len(self.xs)))
+                    self.xs.append(x)
+                    qx, qh = qbuf(Wgu.K), qbuf(I)
+                    h = torch.empty(M, I, dtype=bf, device=dev)
+                    y = torch.empty(M, Wd.N, dtype=bf, device=dev)
+                    self._add_quant(f"amax+quant x{i}", x, Wgu.K, qx)
+                    self.ops.append((f"gemm {lin[i].name}+swiglu", "gemm",
+                                     lambda st, qx=qx, Wgu=Wgu, h=h, qh=qh: qh.__setitem__(
+                                         "n", mq.mq_gemm_nvfp4_swiglu(qx["codes"], qx["sf"], qx["s"], M,
+                                                                      Wgu.handle, h, qh["part"], st))))
+                    self.ops.append((f"quant h{i}", "quant",
+                                     lambda st, h=h, qh=qh, I=I: mq.mq_quantize_nvfp4(
+                                         h, M, I, I, qh["codes"], qh["sf"], qh["s"],
+                                         amax_partials=qh["part"], n_partials=qh["n"], stream=st)))
+                    self.ops.append((f"gemm {lin[i + 1].name}", "gemm",
+                                     lambda st, qh=qh, Wd=Wd, y=y: mq.mq_gemm_nvfp4(
+                                         qh["codes"], qh["sf"], qh["s"], M, Wd.handle, y, Wd.N, st)))
+                    self.flops += 2.0 * M * Wgu.N * Wgu.K + 2.0 * M * Wd.N * Wd.K
+                    i += 2
+                else:
+                    x = workloads.layer_activation(wl, W.K, i, device=str(dev))
+                    self.plan.append(("linear", i, len(self.xs)))
+                    self.xs.append(x)
+                    q = qbuf(W.K)
+                    y = torch.empty(M, W.N, dtype=bf, device=dev)
+                    self._add_quant(f"amax+quant x{i}", x, W.K, q)
+                    self.ops.append((f"gemm {lin[i].name}", "gemm",
+                                     lambda st, q=q, W=W, y=y: mq.mq_gemm_nvfp4(
+                                         q["codes"], q["sf"], q["s"], M, W.handle, y, W.N, st)))
+                    self.flops += 2.0 * M * W.N * W.K
+                    i += 1
         elif wl.chunks > 1:
             # each chunk quantized once and used by every projection
             K = self.W[0].K
@@ -418,11 +440,16 @@ def run_gpu(args, wl, world, rank):
     try:
         def bf16_prefill():
             if wl.swiglu:
-                for i in range(0, len(P.ws), 2):
-                    gu = torch.matmul(P.xs[i // 2], P.ws[i].t())
-                    I = gu.shape[1] // 2
-                    h = torch.nn.functional.silu(gu[:, :I]) * gu[:, I:]
-                    torch.matmul(h, P.ws[i + 1].t())
+                for item in P.plan:
+                    if item[0] == "mlp":
+                        _, i, j, xi = item
+                        gu = torch.matmul(P.xs[xi], P.ws[i].t())
+                        I = gu.shape[1] // 2
+                        h = torch.nn.functional.silu(gu[:, :I]) * gu[:, I:]
+                        torch.matmul(h, P.ws[j].t())
+                    else:
+                        _, i, xi = item
+                        torch.matmul(P.xs[xi], P.ws[i].t())
             elif wl.chunks > 1:
                 for x in P.xs:
                     for w in P.ws:
