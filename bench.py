@@ -295,13 +295,24 @@ class Prefill:
                 self.flops += 2.0 * M * W.N * W.K
         # decode (phase switch) on every weight handle at M = 1
         self.dec = []
-        xdec = self.xs[0][:1]
+        xdec = self.xs[0][:1].contiguous()
         for W in self.W:
             xd = xdec if W.K == xdec.shape[1] else torch.zeros(1, W.K, dtype=bf, device=dev)
             yd = torch.empty(1, W.N, dtype=bf, device=dev)
             self.dec.append(lambda st, W=W, xd=xd, yd=yd: mq.mq_decode_linear_bf16(
                 W.handle, xd, 1, yd, st))
         self.decode_bytes = sum(2.0 * W.N * W.K + 2.0 * W.K + 2.0 * W.N for W in self.W)
+        # uniform-NVFP4 (W4A4) decode on the same handles: x quantized per call
+        self.dec4 = []
+        for W in self.W:
+            xd = xdec if W.K == xdec.shape[1] else torch.zeros(1, W.K, dtype=bf, device=dev)
+            yd = torch.empty(1, W.N, dtype=bf, device=dev)
+            nb = mq.mq_workspace_bytes(1, W.K)
+            ws4 = torch.empty(nb, dtype=torch.uint8, device=dev)
+            self.dec4.append(lambda st, W=W, xd=xd, yd=yd, ws4=ws4, nb=nb: mq.mq_decode_linear_nvfp4(
+                W.handle, xd, 1, yd, ws4, nb, st))
+        # weight codes + E4M3 scales (0.5625 byte per parameter) and x / y
+        self.decode4_bytes = sum(0.5625 * W.N * W.K + 2.0 * W.K + 2.0 * W.N for W in self.W)
         self.launches = len(self.ops) + len(self.dec)   # one kernel per op / decode call
 
     def _add_quant(self, name, x, K, q):
@@ -393,6 +404,20 @@ def run_gpu(args, wl, world, rank):
         flush()
         step_breakdown(bd_evs[k])
     torch.cuda.synchronize()
+    # uniform-NVFP4 decode (M = 1) on the same handles, after an L2 flush
+    d4 = []
+    for _ in range(max(3, min(args.steps, 10))):
+        flush()
+        a, b = ev(), ev()
+        a.record(stream)
+        for f in P.dec4:
+            f(stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        d4.append(a.elapsed_time(b))
+    t_dec4 = statistics.median(d4)
+    if mq.mq_check(stream) != 0:
+        raise RuntimeError("device error during the NVFP4 decode pass")
     per_kind = {"amax": 0.0, "quant": 0.0, "gemm": 0.0}
     per_op = [0.0] * nop
     for evs in bd_evs:
@@ -483,11 +508,33 @@ def run_gpu(args, wl, world, rank):
         wsb = max(mq.mq_workspace_bytes(M, W.K) for W in P.W)
         wsp = torch.empty(wsb, dtype=torch.uint8, device=dev)
 
+        # host->device copies, the prefill and device->host copies on three
+        # streams, so PCIe carries X in and Y out at the same time while the
+        # GPU computes; events keep each buffer's reuse ordered
+        h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+        n_proj = len(P.W)
+        x_ready = [ev() for _ in range(n_proj)]
+        x_free = [ev() for _ in range(n_proj)]
+        y_ready = [ev() for _ in range(n_proj)]
+        y_free = [ev() for _ in range(n_proj)]
+        for e in x_free + y_free:
+            e.record(stream)
+
         def e2e_step():
-            for W, xh, xd, yd, yh in zip(P.W, xs_h, xs_d, ys_d, ys_h):
-                xd.copy_(xh, non_blocking=True)
+            for i, (W, xh, xd, yd, yh) in enumerate(zip(P.W, xs_h, xs_d, ys_d, ys_h)):
+                h2d.wait_event(x_free[i])
+                with torch.cuda.stream(h2d):
+                    xd.copy_(xh, non_blocking=True)
+                x_ready[i].record(h2d)
+                stream.wait_event(x_ready[i])
+                stream.wait_event(y_free[i])
                 mq.mq_prefill_linear_nvfp4(W.handle, xd, M, yd, wsp, wsb, stream)
-                yh.copy_(yd, non_blocking=True)
+                x_free[i].record(stream)
+                y_ready[i].record(stream)
+                d2h.wait_event(y_ready[i])
+                with torch.cuda.stream(d2h):
+                    yh.copy_(yd, non_blocking=True)
+                y_free[i].record(d2h)
 
         for _ in range(2):
             e2e_step()
@@ -497,15 +544,19 @@ def run_gpu(args, wl, world, rank):
         barrier(world)
         torch.cuda.synchronize()
         e0.record(stream)
+        h2d.wait_event(e0)
         for _ in range(n_e2e):
             e2e_step()
+        for e in y_free:
+            stream.wait_event(e)
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = reduce_over_ranks(e0.elapsed_time(e1) / n_e2e, world, "MAX")
         e2e = {"value": round(total_flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                "h2d_bytes_per_step": sum(x.numel() * 2 for x in P.xs),
                "d2h_bytes_per_step": sum(M * W.N * 2 for W in P.W),
-               "path": "mq_prefill_linear_nvfp4, pinned-host X in / Y out, per projection"}
+               "path": "mq_prefill_linear_nvfp4 per projection; pinned-host X in and Y out "
+                       "on their own streams, overlapping each other and the compute"}
 
     traffic, traffic_launches = recorded_traffic(args.workload)
     clk = clocks.summary()
@@ -542,6 +593,10 @@ def run_gpu(args, wl, world, rank):
         "per_launch_ms": {P.ops[i][0]: round(per_op[i] / K_, 4) for i in range(nop)},
         "decode_m1_ms": round(t_dec / K_, 4),
         "decode_gbs": round(P.decode_bytes / (t_dec / K_ * 1e-3) / 1e9, 1),
+        "decode_nvfp4_m1_ms": round(t_dec4, 4),
+        "decode_nvfp4_gbs": round(P.decode4_bytes / (t_dec4 * 1e-3) / 1e9, 1),
+        "decode_nvfp4_note": "W4A4 decode (x quantized per call: amax, quantize, GEMV), "
+                             "separate pass; GB/s over 0.5625 B/param + x + y",
         "graph_prefill_ms": round(graph_ms, 4) if isinstance(graph_ms, float) else graph_ms,
         "tokens_per_s": round(world * wl.M * max(1, wl.chunks) / (t_prefill_max * 1e-3), 1),
         "fp4_peak_frac": round(value / fp4_peak, 4),

@@ -215,6 +215,22 @@ mq_status mq_prefill_linear_nvfp4_noalloc(const mq_weight *w, const void *x_bf16
 mq_status mq_decode_linear_bf16(const mq_weight *w, const void *x_bf16, int64_t M, void *y_bf16,
                                 cudaStream_t stream);
 
+/* Uniform-NVFP4 decode linear (W4A4), the decode half of quantizing both
+ * phases, which the Mix-Quant pages compare their scheme against
+ * (gist.science technical summary, section 1 "Problem Statement" and section
+ * 4 "Experimental Results"): x is quantized with the prefill recipe (one tensor
+ * scale for the call, E4M3 scale per 16, E2M1 codes) into `workspace`, then
+ * y[m, n] = bf16( sum_k deq(xq)[m,k] deq(wq)[n,k] / (s_enc_x s_enc_w) ) on the
+ * handle's NVFP4 copy, FP32 accumulation -- the same arithmetic as
+ * mq_prefill_linear_nvfp4, streaming 0.5625 byte per weight instead of 2.
+ * x (device) BF16 [M, K] contiguous, y (device) BF16 [M, N] contiguous; any
+ * M >= 1, meant for M <= 8.  workspace (device, 256-byte aligned) of at least
+ * mq_workspace_bytes(M, K) bytes.  Shares the handle's split-K scratch with
+ * mq_decode_linear_bf16: decode calls on one handle must not overlap on the
+ * GPU. */
+mq_status mq_decode_linear_nvfp4(const mq_weight *w, const void *x_bf16, int64_t M, void *y_bf16,
+                                 void *workspace, size_t ws_bytes, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

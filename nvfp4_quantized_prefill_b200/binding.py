@@ -38,6 +38,7 @@ SIGNATURES = [
     ("mq_prefill_mlp_swiglu_nvfp4", _I, [_P, _P, _P, _I64, _P, _P, _P, _SZ, _P]),
     ("mq_prefill_linear_nvfp4_noalloc", _I, [_P, _P, _I64, _P, _P]),
     ("mq_decode_linear_bf16", _I, [_P, _P, _I64, _P, _P]),
+    ("mq_decode_linear_nvfp4", _I, [_P, _P, _I64, _P, _P, _SZ, _P]),
 ]
 
 _lib = None
@@ -175,6 +176,12 @@ def mq_prefill_linear_nvfp4_noalloc(weight: int, x, M: int, y, stream=None) -> N
 def mq_decode_linear_bf16(weight: int, x, M: int, y, stream=None) -> None:
     _ok("mq_decode_linear_bf16", lib().mq_decode_linear_bf16(weight, _ptr(x), M, _ptr(y),
                                                              _stream(stream)))
+
+
+def mq_decode_linear_nvfp4(weight: int, x, M: int, y, workspace, ws_bytes: int,
+                           stream=None) -> None:
+    _ok("mq_decode_linear_nvfp4", lib().mq_decode_linear_nvfp4(
+        weight, _ptr(x), M, _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)))
 
 
 class Weight:

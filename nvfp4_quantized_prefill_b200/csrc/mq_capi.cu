@@ -466,6 +466,31 @@ mq_status mq_prefill_linear_nvfp4_noalloc(const mq_weight *w, const void *x_bf16
                      stream);
 }
 
+mq_status mq_decode_linear_nvfp4(const mq_weight *w, const void *x_bf16, int64_t M, void *y_bf16,
+                                 void *workspace, size_t ws_bytes, cudaStream_t stream) {
+    if (!x_bf16 || !y_bf16 || !workspace) return MQ_ERR_INVALID_ARG;
+    mq_status st = check_weight(w);
+    if (st != MQ_OK) return st;
+    if (M < 1 || M > (1LL << 20) || !shape_fits(M, w->K)) return MQ_ERR_SHAPE;
+    if (ws_bytes < act_ws_bytes(M, w->K)) return MQ_ERR_INVALID_ARG;
+    if (!aligned16(x_bf16) || !aligned16(y_bf16) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return MQ_ERR_ALIGNMENT;
+    DeviceInfo *d = nullptr;
+    st = device_info(&d);
+    if (st != MQ_OK) return st;
+    if (M <= 8)  // the kernel quantizes the tokens itself
+        return cuda_status(mq::launch_decode_nvf4(nullptr, nullptr, nullptr, x_bf16, M, w->codes,
+                                                  w->sf, w->s_enc, w->N, w->K, y_bf16,
+                                                  w->decode_scratch, d->num_sms, stream));
+    ActWs a = carve_act(static_cast<uint8_t *>(workspace), M, w->K);
+    st = quantize_impl(d, x_bf16, M, w->K, w->K, a.codes, a.sf, a.s_enc, nullptr, 0, a.partials,
+                       stream);
+    if (st != MQ_OK) return st;
+    return cuda_status(mq::launch_decode_nvf4(a.codes, a.sf, a.s_enc, nullptr, M, w->codes, w->sf,
+                                              w->s_enc, w->N, w->K, y_bf16, w->decode_scratch,
+                                              d->num_sms, stream));
+}
+
 mq_status mq_decode_linear_bf16(const mq_weight *w, const void *x_bf16, int64_t M, void *y_bf16,
                                 cudaStream_t stream) {
     if (!x_bf16 || !y_bf16) return MQ_ERR_INVALID_ARG;

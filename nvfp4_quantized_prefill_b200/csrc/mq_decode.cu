@@ -16,7 +16,8 @@
 // load the FP32 pipes.  K is split into S slices so that there are enough
 // units to balance the SMs; the last CTA of a row group to finish (an atomic
 // counter, reset by that CTA) adds the S partial sums in slice order --
-// deterministically -- and writes BF16.
+// deterministically -- and writes BF16.  Scratch (per weight): one counter per
+// row group first, then the partial sums.
 #include <cuda_bf16.h>
 
 #include "mq_internal.h"
@@ -130,20 +131,27 @@ int decode_slices(int64_t N, int64_t K, int num_sms) {
     return static_cast<int>(S);
 }
 
+size_t decode_counter_bytes(int64_t N) {
+    const int64_t groups = (N + kRows - 1) / kRows;
+    return (static_cast<size_t>(groups) * sizeof(unsigned) + 255) / 256 * 256;
+}
+
 size_t decode_scratch_bytes(int64_t N, int64_t K, int num_sms) {
-    const int S = decode_slices(N, K, num_sms);
+    int S = decode_slices(N, K, num_sms);
+    const int S4 = decode_nvf4_slices(N, K, num_sms);
+    if (S4 > S) S = S4;
     if (S == 1) return 0;
     const int64_t groups = (N + kRows - 1) / kRows;
-    return static_cast<size_t>(groups) * (S * 128 * sizeof(float) + sizeof(unsigned));
+    return decode_counter_bytes(N) + static_cast<size_t>(groups) * S * 128 * sizeof(float);
 }
 
 cudaError_t launch_decode(const void *x, int64_t M, const void *w, int64_t N, int64_t K, void *y,
                           void *scratch, int num_sms, cudaStream_t s) {
     const int S = decode_slices(N, K, num_sms);
     const int64_t groups = (N + kRows - 1) / kRows;
-    float *partials = static_cast<float *>(scratch);
-    unsigned *counters =
-        S > 1 ? reinterpret_cast<unsigned *>(partials + groups * S * 128) : nullptr;
+    unsigned *counters = static_cast<unsigned *>(scratch);
+    float *partials = reinterpret_cast<float *>(static_cast<uint8_t *>(scratch) +
+                                                decode_counter_bytes(N));
     const int grid = static_cast<int>(groups * S);
     for (int64_t m0 = 0; m0 < M; m0 += 8) {
         const int mg = static_cast<int>(M - m0 < 8 ? M - m0 : 8);

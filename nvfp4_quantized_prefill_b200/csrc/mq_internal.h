@@ -87,16 +87,27 @@ bool encode_codes_tmap(CUtensorMap *map, const void *codes, int64_t rows, int64_
 // 256-wide K step of one 128-row block.
 bool encode_sf_tmap(CUtensorMap *map, const void *sf, int64_t rows, int64_t K);
 
-// ---- BF16 decode (mq_decode.cu) ------------------------------------------------
+// ---- decode (mq_decode.cu: BF16; mq_decode_nvf4.cu: NVFP4 W4A4) ----------------
 
-// Number of K slices the decode splits an [N, K] weight into, and the bytes of
-// per-weight scratch it needs for them (0 when S = 1): S x 128 FP32 partial
-// sums and one counter per 16-row group; the counters must start at zero and
-// are left at zero by every launch.
+// Number of K slices the BF16 / NVFP4 decode splits an [N, K] weight into,
+// and the bytes of per-weight scratch they need (0 when both use S = 1): one
+// counter per 16-row group (decode_counter_bytes, at the start; the counters
+// must start at zero and are left at zero by every launch), then S x 128 FP32
+// partial sums per group for the larger S.
 int decode_slices(int64_t N, int64_t K, int num_sms);
+int decode_nvf4_slices(int64_t N, int64_t K, int num_sms);
+size_t decode_counter_bytes(int64_t N);
 size_t decode_scratch_bytes(int64_t N, int64_t K, int num_sms);
 
 cudaError_t launch_decode(const void *x, int64_t M, const void *w, int64_t N, int64_t K,
                           void *y, void *scratch, int num_sms, cudaStream_t s);
+
+// W4A4 decode, weights from the handle's NVFP4 copy.  With x_bf16 set (M <= 8)
+// the kernel quantizes the tokens itself; otherwise x is given quantized
+// (codes, swizzled scales with rows padded to 128, tensor scale).
+cudaError_t launch_decode_nvf4(const uint8_t *x_codes, const uint8_t *x_sf, const float *s_enc_x,
+                               const void *x_bf16, int64_t M, const uint8_t *w_codes,
+                               const uint8_t *w_sf, const float *s_enc_w, int64_t N, int64_t K,
+                               void *y, void *scratch, int num_sms, cudaStream_t s);
 
 }  // namespace mq

@@ -21,6 +21,7 @@
 #include <cuda_fp16.h>
 
 #include "mq_internal.h"
+#include "mq_nvfp4.cuh"
 
 namespace mq {
 
@@ -60,17 +61,6 @@ __device__ __forceinline__ uint4 ldg_v4_stream(const uint4 *p) {
 #else
     return __ldg(p);
 #endif
-}
-
-// max of |bf16| over the 8 values of a 16-byte vector, as 16-bit magnitude bits
-// (non-negative bf16 values order like their bit patterns).
-__device__ __forceinline__ uint32_t absmax8_bits(uint4 v) {
-    uint32_t a, b;
-    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(a) : "r"(v.x), "r"(v.y));
-    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(b) : "r"(v.z), "r"(v.w));
-    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(a) : "r"(a), "r"(b));
-    a &= 0x7FFF7FFFu;
-    return max(a & 0xFFFFu, a >> 16);
 }
 
 __device__ __forceinline__ float block_max(float v, float *red) {
@@ -119,12 +109,6 @@ __global__ void __launch_bounds__(kThreads, kAmaxBlocksPerSm)
     if (threadIdx.x == 0) partials[blockIdx.x] = m;
 }
 
-// E4M3 byte -> float (exact).
-__device__ __forceinline__ float e4m3_to_float(uint32_t b) {
-    __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(b), __NV_E4M3);
-    return __half2float(__half(h));
-}
-
 // Byte offset of the 4 scales (r, 4*cq .. 4*cq+3) in the swizzled layout.
 __device__ __forceinline__ uint64_t sf_word_offset(uint32_t r, uint32_t cq, uint32_t ctiles) {
     return (static_cast<uint64_t>(r >> 7) * ctiles + cq) * 512u + (r & 31u) * 16u +
@@ -133,78 +117,6 @@ __device__ __forceinline__ uint64_t sf_word_offset(uint32_t r, uint32_t cq, uint
 
 constexpr int kQuantUnroll = MQ_QUANT_UNROLL;
 constexpr int kQuantBlocksPerSm = MQ_QUANT_BLOCKS_PER_SM;
-
-// fp32(a / 6) for a non-negative finite BF16 value a, in three operations:
-// q0 = RN(a * RN(1/6)), r = RN(a - 6 q0) (exact by FMA), q = RN(r * RN(1/6) + q0).
-// Checked exhaustively against IEEE division for all 32640 non-negative finite
-// BF16 inputs.
-__device__ __forceinline__ float div6_bf16(float a) {
-    const float inv6 = 0.16666667163372039794921875f;  // RN(1/6)
-    const float q0 = __fmul_rn(a, inv6);
-    const float r = __fmaf_rn(-q0, 6.0f, a);
-    return __fmaf_rn(r, inv6, q0);
-}
-
-// max(|a|, |b|) per BF16 half, sign bits = sign(a) ^ sign(b) (mask them off
-// to read the magnitudes).
-__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-
-// Eight BF16 values (two per word, element 2j in the low half of word j)
-// times f, each product rounded to FP32 (packed f32x2 multiplies) and then to
-// E2M1 (round-to-nearest-even, saturating at 6, the sign of x kept even when
-// the code is zero); returns the four code bytes, element 2j in the low
-// nibble of byte j.
-__device__ __forceinline__ uint32_t e2m1x8(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3,
-                                           float f) {
-    uint32_t out;
-    asm("{\n\t"
-        ".reg .b8 c0, c1, c2, c3;\n\t"
-        ".reg .b64 f2, x0, x1, x2, x3;\n\t"
-        ".reg .b32 l0, h0, l1, h1, l2, h2, l3, h3;\n\t"
-        "mov.b64 f2, {%5, %5};\n\t"
-        "shl.b32 l0, %1, 16;\n\tand.b32 h0, %1, 0xFFFF0000;\n\t"
-        "shl.b32 l1, %2, 16;\n\tand.b32 h1, %2, 0xFFFF0000;\n\t"
-        "shl.b32 l2, %3, 16;\n\tand.b32 h2, %3, 0xFFFF0000;\n\t"
-        "shl.b32 l3, %4, 16;\n\tand.b32 h3, %4, 0xFFFF0000;\n\t"
-        "mov.b64 x0, {l0, h0};\n\tmov.b64 x1, {l1, h1};\n\t"
-        "mov.b64 x2, {l2, h2};\n\tmov.b64 x3, {l3, h3};\n\t"
-        "mul.rn.f32x2 x0, x0, f2;\n\tmul.rn.f32x2 x1, x1, f2;\n\t"
-        "mul.rn.f32x2 x2, x2, f2;\n\tmul.rn.f32x2 x3, x3, f2;\n\t"
-        "mov.b64 {l0, h0}, x0;\n\tmov.b64 {l1, h1}, x1;\n\t"
-        "mov.b64 {l2, h2}, x2;\n\tmov.b64 {l3, h3}, x3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 c0, h0, l0;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 c1, h1, l1;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 c2, h2, l2;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 c3, h3, l3;\n\t"
-        "mov.b32 %0, {c0, c1, c2, c3};\n\t"
-        "}"
-        : "=r"(out)
-        : "r"(w0), "r"(w1), "r"(w2), "r"(w3), "f"(f));
-    return out;
-}
-
-// One lane quantizes one 16-element block held in w[0..7] (two BF16 per word,
-// element 2j in the low half of w[j]).  ftab[b] = s_enc / dec(b) for every
-// non-negative E4M3 byte b (0 for b = 0).  Returns the 8 code bytes in (lo, hi)
-// and the block scale byte in *sb_out.
-__device__ __forceinline__ void quantize_block16(const uint32_t (&w)[8], float s_enc,
-                                                 const float *ftab, uint32_t &lo, uint32_t &hi,
-                                                 uint32_t &sb_out) {
-    uint32_t a = absmax_bf16x2(absmax_bf16x2(absmax_bf16x2(w[0], w[1]), absmax_bf16x2(w[2], w[3])),
-                               absmax_bf16x2(absmax_bf16x2(w[4], w[5]), absmax_bf16x2(w[6], w[7])));
-    a &= 0x7FFF7FFFu;
-    const float amax_b = __uint_as_float(max(a & 0xFFFFu, a >> 16) << 16);
-    const float sbf = __fmul_rn(div6_bf16(amax_b), s_enc);
-    const uint32_t sb = __nv_cvt_float_to_fp8(sbf, __NV_SATFINITE, __NV_E4M3);
-    const float f = ftab[sb];  // = dec(sb) == 0 ? 0 : fp32(s_enc / dec(sb))
-    lo = e2m1x8(w[0], w[1], w[2], w[3], f);
-    hi = e2m1x8(w[4], w[5], w[6], w[7], f);
-    sb_out = sb;
-}
 
 // Each warp quantizes 512-element row segments (lane l: 16-block l of the
 // segment, two 16-byte loads), kQuantUnroll segments per iteration with all
@@ -222,13 +134,9 @@ __global__ void __launch_bounds__(kThreads, kQuantBlocksPerSm) quantize_kernel(
 #pragma unroll 4
     for (int i = threadIdx.x; i < n_partials; i += kThreads) amx = fmaxf(amx, partials[i]);
     const float amax = block_max(amx, red);
-    float s_enc = __fdiv_rn(2688.0f, amax);
-    if (amax == 0.0f || !isfinite(s_enc)) s_enc = 1.0f;
+    const float s_enc = nvfp4_tensor_scale(amax);
     if (blockIdx.x == 0 && threadIdx.x == 0) *s_enc_out = s_enc;
-    if (threadIdx.x < 128) {
-        const float dec = e4m3_to_float(threadIdx.x);
-        ftab[threadIdx.x] = dec == 0.0f ? 0.0f : __fdiv_rn(s_enc, dec);
-    }
+    nvfp4_scale_table(s_enc, ftab);
     __syncthreads();
 
     const uint32_t ctiles = K / 64u;
@@ -279,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, kQuantBlocksPerSm) quantize_kernel(
 #pragma unroll
         for (int u = 0; u < kQuantUnroll; ++u) {
             uint32_t lo, hi, sb;
-            quantize_block16(w[u], s_enc, ftab, lo, hi, sb);
+            quantize_block16<true>(w[u], s_enc, ftab, lo, hi, sb);
             const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sb, 1);
             const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sb, 2);
             const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sb, 3);
