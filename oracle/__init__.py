@@ -75,6 +75,10 @@ def _load():
             lib.mqo_decode_linear.argtypes = [P, I64, P, I64, I64, P, P]
             lib.mqo_swiglu.restype = None
             lib.mqo_swiglu.argtypes = [P, P, I64, P]
+            lib.mqo_double_to_bf16_rne.restype = ctypes.c_uint16
+            lib.mqo_double_to_bf16_rne.argtypes = [ctypes.c_double]
+            lib.mqo_rmsnorm.restype = None
+            lib.mqo_rmsnorm.argtypes = [P, I64, I64, I64, P, ctypes.c_double, P]
             lib.mqo_set_threads.restype = None
             lib.mqo_set_threads.argtypes = [ctypes.c_int]
             lib.mqo_threads_used.restype = ctypes.c_int
@@ -249,3 +253,20 @@ def swiglu(g, u) -> np.ndarray:
     h = np.zeros(ga.shape, dtype=np.uint16)
     _load().mqo_swiglu(_ptr(ga), _ptr(ua), ga.size, _ptr(h))
     return h
+
+
+def double_to_bf16(v: float) -> int:
+    """One binary64 -> BF16 round-to-nearest-even; returns the bit pattern."""
+    return int(_load().mqo_double_to_bf16_rne(float(v)))
+
+
+def rmsnorm(x, gamma, eps: float) -> np.ndarray:
+    """y = bf16(gamma * bf16(x / sqrt(mean(x^2) + eps))) per row, binary64
+    (the RMSNorm in front of a prefill linear); returns uint16 bf16 bits."""
+    xa = _u16(x)
+    ga = _u16(gamma)
+    rows, cols = xa.shape
+    assert ga.shape == (cols,)
+    y = np.zeros((rows, cols), dtype=np.uint16)
+    _load().mqo_rmsnorm(_ptr(xa), rows, cols, cols, _ptr(ga), float(eps), _ptr(y))
+    return y

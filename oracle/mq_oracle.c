@@ -357,3 +357,52 @@ void mqo_swiglu(const uint16_t *g, const uint16_t *u, int64_t n, uint16_t *h) {
         h[i] = mqo_float_to_bf16_rne(hv);
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* RMSNorm in front of a prefill linear                                     */
+/* ------------------------------------------------------------------------ */
+
+/* Round a binary64 value to the nearest BF16 (ties to even), directly --
+ * not through binary32, so there is one rounding. */
+uint16_t mqo_double_to_bf16_rne(double v) {
+    if (v == 0.0) return signbit(v) ? 0x8000u : 0u;
+    if (isnan(v)) return 0x7FC0u;
+    const int neg = v < 0.0;
+    double a = neg ? -v : v;
+    if (isinf(a)) return (uint16_t)(neg ? 0xFF80u : 0x7F80u);
+    int e;
+    (void)frexp(a, &e);              /* a = m 2^e, 0.5 <= m < 1 */
+    int ulp_exp = e - 8;             /* 8 significant bits */
+    if (ulp_exp < -133) ulp_exp = -133; /* BF16 subnormal spacing 2^-133 */
+    double q = rint(ldexp(a, -ulp_exp)); /* round half to even */
+    double r = ldexp(q, ulp_exp);
+    if (r > 3.38953138925153547590470800371487866880e+38) return (uint16_t)(neg ? 0xFF80u : 0x7F80u);
+    uint16_t b = mqo_float_to_bf16_rne((float)r);  /* exact: r has <= 8 significant bits */
+    return (uint16_t)(neg ? (b | 0x8000u) : b);
+}
+
+/* [reading] The pages do not define the normalisation that produces the
+ * prefill linear's input (the step before the QKV and gate/up projections);
+ * the Llama-family RMSNorm is used, evaluated in binary64 from the BF16 row x
+ * and BF16 gain gamma:
+ *   r   = 1 / sqrt( sum_k x_k^2 / K + eps )
+ *   t_k = bf16_RNE(x_k * r)          (the normalised row in the input type)
+ *   y_k = bf16_RNE(gamma_k * t_k)    (the learned per-channel gain)        */
+void mqo_rmsnorm(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, const uint16_t *gamma,
+                 double eps, uint16_t *y) {
+#pragma omp parallel for schedule(static) num_threads(MQO_NT)
+    for (int64_t m = 0; m < rows; ++m) {
+        const uint16_t *xr = x + m * ld;
+        double ss = 0.0;
+        for (int64_t k = 0; k < cols; ++k) {
+            double v = (double)mqo_bf16_to_float(xr[k]);
+            ss += v * v;
+        }
+        double r = 1.0 / sqrt(ss / (double)cols + eps);
+        for (int64_t k = 0; k < cols; ++k) {
+            double t = (double)mqo_bf16_to_float(mqo_double_to_bf16_rne((double)mqo_bf16_to_float(xr[k]) * r));
+            double gk = (double)mqo_bf16_to_float(gamma[k]);
+            y[m * cols + k] = mqo_double_to_bf16_rne(gk * t);
+        }
+    }
+}

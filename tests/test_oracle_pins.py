@@ -343,3 +343,58 @@ def test_swiglu_against_torch_silu(oracle_mod):
     assert (oracle_mod.swiglu(z, one) == 0).all()
     big = torch.full((1, 8), 30.0, dtype=torch.bfloat16)
     assert (oracle_mod.swiglu(big, one) == bf16_bits(big)).all()   # SiLU(30) ~ 30
+
+
+# ---- RMSNorm in front of a prefill linear (reading: Llama-family RMSNorm) ----
+
+def test_double_to_bf16_matches_torch(oracle_mod):
+    rng = np.random.default_rng(11)
+    vals = np.concatenate([rng.standard_normal(2000) * 10.0 ** rng.integers(-30, 30, 2000),
+                           [0.0, -0.0, 1.0, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -9, 2.0 ** -133,
+                            2.0 ** -134 * 3, 3.0e38, -1.5e-40]])
+    got = np.array([oracle_mod.double_to_bf16(v) for v in vals], dtype=np.uint16)
+    ref = bf16_bits(torch.tensor(vals, dtype=torch.float64).to(torch.bfloat16))
+    assert (got == ref).all()
+
+
+def test_rmsnorm_closed_forms(oracle_mod):
+    K = 64
+    # constant rows: x / |x| exactly (eps = 0), with gain 1
+    cs = [3.0, -0.75, 1e-3, -250.0, 2.0 ** -20]
+    x = torch.tensor([[c] * K for c in cs], dtype=torch.bfloat16)
+    one = torch.ones(K, dtype=torch.bfloat16)
+    y = oracle_mod.rmsnorm(x, one, 0.0)
+    exp = bf16_bits(torch.tensor([[math.copysign(1.0, c)] * K for c in cs], dtype=torch.bfloat16))
+    assert (y == exp).all()
+    # one-hot rows of length 4: x_j / sqrt(x_j^2 / 4) = 2 sign(x_j); gain scales it
+    x4 = torch.zeros(3, 4, dtype=torch.bfloat16)
+    x4[0, 1] = 5.0
+    x4[1, 3] = -0.125
+    x4[2, 0] = 77.0
+    g4 = torch.tensor([0.5, -1.5, 3.0, 0.25], dtype=torch.bfloat16)
+    y4 = torch.from_numpy(oracle_mod.rmsnorm(x4, g4, 0.0).view(np.int16)).view(torch.bfloat16).float()
+    exp4 = torch.zeros(3, 4)
+    exp4[0, 1] = 2.0 * -1.5
+    exp4[1, 3] = -2.0 * 0.25
+    exp4[2, 0] = 2.0 * 0.5
+    assert torch.equal(y4, exp4)
+    # an all-zero row stays zero
+    z = oracle_mod.rmsnorm(torch.zeros(1, K, dtype=torch.bfloat16), one, 1e-5)
+    assert (z & 0x7FFF == 0).all()
+
+
+def test_rmsnorm_scale_invariance(oracle_mod):
+    x = workloads.activation("channel_gain", 16, 256, 12, 0)
+    g = workloads.activation("outlier", 1, 256, 12, 1)[0]
+    y = oracle_mod.rmsnorm(x, g, 0.0)
+    for k in (-3, 5):
+        assert (oracle_mod.rmsnorm((x.float() * 2.0 ** k).to(torch.bfloat16), g, 0.0) == y).all()
+
+
+def test_rmsnorm_matches_torch_library(oracle_mod):
+    """Unit gain: the normalised row is torch's binary64 rms_norm rounded to BF16."""
+    x = workloads.activation("student_t3", 32, 512, 13, 0)
+    one = torch.ones(512, dtype=torch.bfloat16)
+    y = oracle_mod.rmsnorm(x, one, 1e-5)
+    ref = torch.nn.functional.rms_norm(x.double(), (512,), eps=1e-5).to(torch.bfloat16)
+    assert (y == bf16_bits(ref)).all()
