@@ -38,6 +38,7 @@ sys.path.insert(0, ROOT)
 from nvfp4_quantized_prefill_b200 import workloads  # noqa: E402
 
 FP4_OVER_BF16 = 4.0   # nominal dense ratio (9 PF fp4 / 2.25 PF bf16)
+RMS_EPS = 1e-5
 METRIC = "prefill linear TFLOPS (NVFP4 incl. act-quant) and % of B200 dense FP4 peak"
 CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -283,12 +284,30 @@ class Prefill:
                     self.flops += 2.0 * M * W.N * W.K
         else:
             self.xs = []
+            self.rs = []
             for i, (W, lin) in enumerate(zip(self.W, wl.linears)):
-                x = workloads.layer_activation(wl, W.K, i, device=str(dev))
-                self.xs.append(x)
                 q = qbuf(W.K)
                 y = torch.empty(M, W.N, dtype=bf, device=dev)
-                self._add_quant(f"amax+quant x{i}", x, W.K, q)
+                if wl.rmsnorm and i == 0:
+                    # RMSNorm of the residual stream writes x and its amax
+                    r = workloads.layer_activation(wl, W.K, i, device=str(dev))
+                    gain = workloads.rmsnorm_gain(W.K, wl.seed, 50, device=str(dev))
+                    x = torch.empty(M, W.K, dtype=bf, device=dev)
+                    self.rs.append((r, gain))
+                    self.xs.append(x)
+
+                    def rms(st, r=r, gain=gain, x=x, q=q, K=W.K):
+                        q["n"] = mq.mq_rmsnorm_amax(r, gain, RMS_EPS, M, K, K, x, q["part"], st)
+
+                    self.ops.append((f"rmsnorm+amax x{i}", "amax", rms))
+                    self.ops.append((f"quant x{i}", "quant",
+                                     lambda st, x=x, q=q, K=W.K: mq.mq_quantize_nvfp4(
+                                         x, M, K, K, q["codes"], q["sf"], q["s"],
+                                         amax_partials=q["part"], n_partials=q["n"], stream=st)))
+                else:
+                    x = workloads.layer_activation(wl, W.K, i, device=str(dev))
+                    self.xs.append(x)
+                    self._add_quant(f"amax+quant x{i}", x, W.K, q)
                 self.ops.append((f"gemm {lin.name}", "gemm",
                                  lambda st, q=q, W=W, y=y: mq.mq_gemm_nvfp4(
                                      q["codes"], q["sf"], q["s"], M, W.handle, y, W.N, st)))
@@ -480,7 +499,10 @@ def run_gpu(args, wl, world, rank):
                     for w in P.ws:
                         torch.matmul(x, w.t())
             else:
-                for x, w in zip(P.xs, P.ws):
+                for i, (x, w) in enumerate(zip(P.xs, P.ws)):
+                    if wl.rmsnorm and i == 0:
+                        r, gain = P.rs[0]
+                        x = torch.nn.functional.rms_norm(r, (r.shape[1],), weight=gain, eps=RMS_EPS)
                     torch.matmul(x, w.t())
         bf16_prefill()
         bt = []
@@ -496,10 +518,40 @@ def run_gpu(args, wl, world, rank):
     except Exception as e:
         bf16_ms = None
 
+    # ---- RMSNorm-fed linear: the same chain with torch's RMSNorm and a
+    # separate amax pass (what the fused RMSNorm + amax replaces)
+    unfused_ms = None
+    if wl.rmsnorm:
+        r, gain = P.rs[0]
+        W0 = P.W[0]
+        qu = dict(codes=torch.empty(wl.M, W0.K // 2, dtype=torch.uint8, device=dev),
+                  sf=torch.empty(mq.mq_sf_bytes(wl.M, W0.K), dtype=torch.uint8, device=dev),
+                  s=torch.empty(1, dtype=torch.float32, device=dev),
+                  part=torch.empty(mq.MQ_AMAX_PARTIALS_MAX, dtype=torch.float32, device=dev))
+        yu = torch.empty(wl.M, W0.N, dtype=torch.bfloat16, device=dev)
+
+        def unfused():
+            xu = torch.nn.functional.rms_norm(r, (W0.K,), weight=gain, eps=RMS_EPS)
+            n = mq.mq_tensor_amax(xu, wl.M, W0.K, W0.K, qu["part"], stream)
+            mq.mq_quantize_nvfp4(xu, wl.M, W0.K, W0.K, qu["codes"], qu["sf"], qu["s"],
+                                 amax_partials=qu["part"], n_partials=n, stream=stream)
+            mq.mq_gemm_nvfp4(qu["codes"], qu["sf"], qu["s"], wl.M, W0.handle, yu, W0.N, stream)
+        unfused()
+        ut = []
+        for _ in range(max(3, min(args.steps, 10))):
+            flush()
+            a, b = ev(), ev()
+            a.record(stream)
+            unfused()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ut.append(a.elapsed_time(b))
+        unfused_ms = statistics.median(ut)
+
     # ---- end to end through the public call: pinned host X -> device, prefill
     # linear (amax + quantize + GEMM inside), result back to pinned host memory
     e2e = None
-    if not wl.swiglu and wl.chunks == 1:
+    if not wl.swiglu and wl.chunks == 1 and not wl.rmsnorm:
         M = wl.M
         xs_h = [x.cpu().pin_memory() for x in P.xs]
         ys_h = [torch.empty(M, W.N, dtype=torch.bfloat16).pin_memory() for W in P.W]
@@ -603,6 +655,9 @@ def run_gpu(args, wl, world, rank):
         "gemm_only_tflops": round(achieved, 2),
         "bf16_cublas_ms": round(bf16_ms, 4) if bf16_ms else None,
         "speedup_vs_bf16": round(bf16_ms / t_prefill_ms, 3) if bf16_ms else None,
+        **({"unfused_rmsnorm_ms": round(unfused_ms, 4),
+            "unfused_note": "torch RMSNorm, then amax, quantize, GEMM (the separate amax pass "
+                            "that the fused RMSNorm + amax removes)"} if unfused_ms else {}),
         "roofline": {
             "kernel": "gemm_nvf4_kernel (tcgen05.mma.cta_group::2 kind::mxf4nvf4 block16)",
             "bound": "tensor",
@@ -667,7 +722,7 @@ def main():
 
     world, rank, local = dist_setup()
     out, P = run_gpu(args, wl, world, rank)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not wl.swiglu and wl.chunks == 1:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not wl.swiglu and wl.chunks == 1 and not wl.rmsnorm:
         import oracle
         xs_cpu = [x.cpu() for x in P.xs]
         ws_cpu = [w.cpu() for w in P.ws]

@@ -204,6 +204,37 @@ mq_status mq_prefill_mlp_swiglu_nvfp4(const mq_weight *w_gate_up, const mq_weigh
 mq_status mq_prefill_linear_nvfp4_noalloc(const mq_weight *w, const void *x_bf16, int64_t M,
                                           void *y_bf16, cudaStream_t stream);
 
+/* ---- RMSNorm in front of a prefill linear ----------------------------------
+ * Mix-Quant converts activations to NVFP4 at the phase boundary (zingnex.cn
+ * forum thread, section "动态精度切换") with one tensor scale from the
+ * tensor's amax (gist.science technical summary, section 2 "Hybrid Precision
+ * Strategy").  The QKV and gate/up inputs of a transformer layer come out of
+ * an RMSNorm; the pages do not define it, the Llama family's is used:
+ *   y = bf16( gamma * bf16( x / sqrt(mean(x^2) + eps) ) ) per row (binary32
+ *   sum of squares in a fixed order, correctly rounded reciprocal root).
+ * Emitting the amax of y on the way out removes the quantizer's own amax pass
+ * over the activations. */
+
+/* x (device) BF16 [M, K] (leading dimension ldx, ldx % 8 == 0, K % 8 == 0),
+ * gamma (device) BF16 [K], eps >= 0.  Writes y (device, BF16 [M, K]
+ * contiguous) and *n_partials partial maxima of |y| to amax_partials (device,
+ * MQ_AMAX_PARTIALS_MAX floats are always enough), ready for
+ * mq_quantize_nvfp4.  *n_partials is set on the host at once. */
+mq_status mq_rmsnorm_amax(const void *x_bf16, const void *gamma_bf16, float eps, int64_t M,
+                          int64_t K, int64_t ldx, void *y_bf16, float *amax_partials,
+                          int *n_partials, cudaStream_t stream);
+
+/* Prefill linear fed by an RMSNorm: xn = RMSNorm(r) * gamma (written to xn,
+ * device BF16 [M, K] contiguous, K = the handle's K) with its amax, NVFP4
+ * quantization of xn, block-scaled GEMM with the handle's NVFP4 weight into
+ * y (device, BF16 [M, N] contiguous).  r (device) BF16 [M, K] contiguous,
+ * gamma (device) BF16 [K].  workspace (device, 256-byte aligned) of at least
+ * mq_workspace_bytes(M, K) bytes. */
+mq_status mq_prefill_linear_rmsnorm_nvfp4(const mq_weight *w, const void *r_bf16,
+                                          const void *gamma_bf16, float eps, int64_t M,
+                                          void *xn_bf16, void *y_bf16, void *workspace,
+                                          size_t ws_bytes, cudaStream_t stream);
+
 /* ---- decode (gist.science §2: decoding keeps BF16) ----------------------- */
 
 /* BF16 decode linear on the handle's BF16 copy: y[m, n] = bf16( sum_k x[m,k]

@@ -39,6 +39,8 @@ SIGNATURES = [
     ("mq_prefill_linear_nvfp4_noalloc", _I, [_P, _P, _I64, _P, _P]),
     ("mq_decode_linear_bf16", _I, [_P, _P, _I64, _P, _P]),
     ("mq_decode_linear_nvfp4", _I, [_P, _P, _I64, _P, _P, _SZ, _P]),
+    ("mq_rmsnorm_amax", _I, [_P, _P, ctypes.c_float, _I64, _I64, _I64, _P, _P, ctypes.POINTER(_I), _P]),
+    ("mq_prefill_linear_rmsnorm_nvfp4", _I, [_P, _P, _P, ctypes.c_float, _I64, _P, _P, _P, _SZ, _P]),
 ]
 
 _lib = None
@@ -182,6 +184,23 @@ def mq_decode_linear_nvfp4(weight: int, x, M: int, y, workspace, ws_bytes: int,
                            stream=None) -> None:
     _ok("mq_decode_linear_nvfp4", lib().mq_decode_linear_nvfp4(
         weight, _ptr(x), M, _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def mq_rmsnorm_amax(x, gamma, eps: float, M: int, K: int, ldx: int, y, amax_partials,
+                    stream=None) -> int:
+    """Returns the number of partial maxima written."""
+    n = ctypes.c_int()
+    _ok("mq_rmsnorm_amax", lib().mq_rmsnorm_amax(
+        _ptr(x), _ptr(gamma), float(eps), M, K, ldx, _ptr(y), _ptr(amax_partials),
+        ctypes.byref(n), _stream(stream)))
+    return n.value
+
+
+def mq_prefill_linear_rmsnorm_nvfp4(weight: int, r, gamma, eps: float, M: int, xn, y, workspace,
+                                    ws_bytes: int, stream=None) -> None:
+    _ok("mq_prefill_linear_rmsnorm_nvfp4", lib().mq_prefill_linear_rmsnorm_nvfp4(
+        weight, _ptr(r), _ptr(gamma), float(eps), M, _ptr(xn), _ptr(y), _ptr(workspace), ws_bytes,
+        _stream(stream)))
 
 
 class Weight:

@@ -6,6 +6,7 @@
 // stored once in a form that serves both phases -- here a handle holding the
 // BF16 matrix for decode and its NVFP4 copy for prefill -- and activations are
 // converted (quantized) at the phase boundary on every prefill call.
+#include <cmath>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -369,6 +370,54 @@ mq_status mq_prefill_linear_nvfp4(const mq_weight *w, const void *x_bf16, int64_
     if (st != MQ_OK) return st;
     ActWs a = carve_act(static_cast<uint8_t *>(workspace), M, w->K);
     st = quantize_impl(d, x_bf16, M, w->K, w->K, a.codes, a.sf, a.s_enc, nullptr, 0, a.partials,
+                       stream);
+    if (st != MQ_OK) return st;
+    return gemm_impl(d, a.codes, a.sf, a.s_enc, M, w, y_bf16, w->N, false, nullptr, nullptr,
+                     stream);
+}
+
+mq_status mq_rmsnorm_amax(const void *x_bf16, const void *gamma_bf16, float eps, int64_t M,
+                          int64_t K, int64_t ldx, void *y_bf16, float *amax_partials,
+                          int *n_partials, cudaStream_t stream) {
+    if (!x_bf16 || !gamma_bf16 || !y_bf16 || !amax_partials || !n_partials)
+        return MQ_ERR_INVALID_ARG;
+    if (!(eps >= 0.0f) || !isfinite(eps)) return MQ_ERR_INVALID_ARG;
+    if (M < 1 || K < 8 || K % 8 != 0 || ldx < K || !shape_fits(M, K < 64 ? 64 : K))
+        return MQ_ERR_SHAPE;
+    if (ldx % 8 != 0 || !aligned16(x_bf16) || !aligned16(gamma_bf16) || !aligned16(y_bf16) ||
+        !aligned16(amax_partials))
+        return MQ_ERR_ALIGNMENT;
+    DeviceInfo *d = nullptr;
+    mq_status st = device_info(&d);
+    if (st != MQ_OK) return st;
+    const int g = mq::rmsnorm_grid(M, K, d->num_sms);
+    *n_partials = g;
+    return cuda_status(mq::launch_rmsnorm_amax(x_bf16, M, K, ldx, gamma_bf16, eps, y_bf16,
+                                               amax_partials, g, stream));
+}
+
+mq_status mq_prefill_linear_rmsnorm_nvfp4(const mq_weight *w, const void *r_bf16,
+                                          const void *gamma_bf16, float eps, int64_t M,
+                                          void *xn_bf16, void *y_bf16, void *workspace,
+                                          size_t ws_bytes, cudaStream_t stream) {
+    if (!r_bf16 || !gamma_bf16 || !xn_bf16 || !y_bf16 || !workspace) return MQ_ERR_INVALID_ARG;
+    if (!(eps >= 0.0f) || !isfinite(eps)) return MQ_ERR_INVALID_ARG;
+    mq_status st = check_weight(w);
+    if (st != MQ_OK) return st;
+    if (M < 1 || !shape_fits(M, w->K)) return MQ_ERR_SHAPE;
+    if (ws_bytes < act_ws_bytes(M, w->K)) return MQ_ERR_INVALID_ARG;
+    if (!aligned16(r_bf16) || !aligned16(gamma_bf16) || !aligned16(xn_bf16) || !aligned16(y_bf16) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return MQ_ERR_ALIGNMENT;
+    DeviceInfo *d = nullptr;
+    st = device_info(&d);
+    if (st != MQ_OK) return st;
+    ActWs a = carve_act(static_cast<uint8_t *>(workspace), M, w->K);
+    const int g = mq::rmsnorm_grid(M, w->K, d->num_sms);
+    cudaError_t e = mq::launch_rmsnorm_amax(r_bf16, M, w->K, w->K, gamma_bf16, eps, xn_bf16,
+                                            a.partials, g, stream);
+    if (e != cudaSuccess) return MQ_ERR_CUDA;
+    st = quantize_impl(d, xn_bf16, M, w->K, w->K, a.codes, a.sf, a.s_enc, a.partials, g, nullptr,
                        stream);
     if (st != MQ_OK) return st;
     return gemm_impl(d, a.codes, a.sf, a.s_enc, M, w, y_bf16, w->N, false, nullptr, nullptr,

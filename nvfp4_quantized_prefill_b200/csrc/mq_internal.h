@@ -59,6 +59,16 @@ cudaError_t launch_quantize(const void *x, int64_t M, int64_t K, int64_t ldx,
                             const float *partials, int n_partials, uint8_t *codes,
                             uint8_t *sf_swizzled, float *s_enc, int num_sms, cudaStream_t s);
 
+// ---- RMSNorm with the amax of its output (mq_rmsnorm.cu) ----------------------
+
+// Number of CTAs (= partial maxima) the RMSNorm kernel uses for M rows.
+int rmsnorm_grid(int64_t M, int64_t K, int num_sms);
+
+// y = RMSNorm(x) * gamma (BF16 [M, K] contiguous) and `grid` partial maxima of
+// |y|; x BF16 [M, K] with leading dimension ldx, gamma BF16 [K].
+cudaError_t launch_rmsnorm_amax(const void *x, int64_t M, int64_t K, int64_t ldx, const void *gamma,
+                                float eps, void *y, float *partials, int grid, cudaStream_t s);
+
 // ---- block-scaled GEMM (mq_gemm.cu) ------------------------------------------
 
 struct GemmArgs {

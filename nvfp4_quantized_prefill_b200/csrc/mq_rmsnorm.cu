@@ -1,0 +1,122 @@
+// mq_rmsnorm.cu -- RMSNorm in front of a prefill linear, emitting the amax of
+// its output for the NVFP4 quantizer.
+//
+// Method: Mix-Quant converts activations to NVFP4 at the phase boundary
+// (zingnex.cn forum thread, section "动态精度切换"), with one tensor-level
+// scale from the tensor's absolute maximum (gist.science technical summary,
+// section 2 "Hybrid Precision Strategy").  In a transformer layer the QKV and
+// gate/up inputs come out of an RMSNorm, so the kernel that writes them can
+// take that maximum on the way out -- the quantizer then skips its own pass
+// over the activations.  RMSNorm (the pages do not define it; the Llama
+// family's is used):
+//   r   = RN(1 / sqrt(RN(sum_k x_k^2 / K) + eps))   (binary32)
+//   t_k = bf16_RNE(x_k * r),  y_k = bf16_RNE(gamma_k * t_k).
+// The sum of squares is taken in binary32 in a fixed order (lane-strided
+// partial sums, then a butterfly), so the result is deterministic; it can
+// differ from the binary64 definition by an ulp of r, which moves a t_k by
+// one BF16 step in rare cases.
+//
+// One warp per row, persistent over rows: a first pass over the row's 16-byte
+// vectors sums the squares, a second reads the row again (L1 / L2), writes y
+// and keeps max|y|; each CTA writes one partial maximum.  (Holding a 4096-wide
+// row in registers between the passes needs ~180 registers a thread and one
+// CTA per SM, and measured slower.)
+#include <cuda_bf16.h>
+
+#include "mq_internal.h"
+
+namespace mq {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+__device__ __forceinline__ float lo_f(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float hi_f(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// y pair from an x pair and a gamma pair: bf16(gamma * bf16(x * r)) each half;
+// returns the packed BF16 pair.
+__device__ __forceinline__ uint32_t norm_pair(uint32_t xw, uint32_t gw, float r) {
+    const float t0 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(lo_f(xw), r)));
+    const float t1 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(hi_f(xw), r)));
+    const __nv_bfloat162 y = __floats2bfloat162_rn(__fmul_rn(lo_f(gw), t0), __fmul_rn(hi_f(gw), t1));
+    return *reinterpret_cast<const uint32_t *>(&y);
+}
+
+__global__ void __launch_bounds__(kThreads) rmsnorm_amax_kernel(
+    const uint4 *__restrict__ x, uint32_t M, uint32_t vpr, uint64_t ldv,
+    const uint4 *__restrict__ gamma, float eps, uint4 *__restrict__ y,
+    float *__restrict__ partials) {
+    __shared__ float red[kWarps];
+    griddep_wait();
+    griddep_launch_dependents();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t nwarps = gridDim.x * kWarps;
+    const float kf = static_cast<float>(vpr * 8u);
+    uint32_t mx = 0;  // max |y| as BF16 magnitude bits
+    auto sumsq = [&](const uint4 &q, float ss) {
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            ss = __fmaf_rn(lo_f(w[j]), lo_f(w[j]), ss);
+            ss = __fmaf_rn(hi_f(w[j]), hi_f(w[j]), ss);
+        }
+        return ss;
+    };
+    // writes the y vector, returns its max |y| as BF16 magnitude bits
+    auto emit = [&](const uint4 &q, uint32_t v, float r, uint4 *yr) -> uint32_t {
+        const uint4 g = __ldg(gamma + v);
+        uint4 o;
+        o.x = norm_pair(q.x, g.x, r);
+        o.y = norm_pair(q.y, g.y, r);
+        o.z = norm_pair(q.z, g.z, r);
+        o.w = norm_pair(q.w, g.w, r);
+        yr[v] = o;
+        const uint32_t m4 = 0x7FFF7FFFu;
+        uint32_t a = __vmaxu2(__vmaxu2(o.x & m4, o.y & m4), __vmaxu2(o.z & m4, o.w & m4));
+        a = __vmaxu2(a, a >> 16);
+        return a & 0xFFFFu;
+    };
+    for (uint32_t row = blockIdx.x * kWarps + warp; row < M; row += nwarps) {
+        const uint4 *xr = x + row * ldv;
+        uint4 *yr = y + static_cast<uint64_t>(row) * vpr;
+        float ss = 0.0f;
+#pragma unroll 8
+        for (uint32_t v = lane; v < vpr; v += 32) ss = sumsq(__ldg(xr + v), ss);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xFFFFFFFFu, ss, o));
+        const float r = __frsqrt_rn(__fadd_rn(__fdiv_rn(ss, kf), eps));
+#pragma unroll 4
+        for (uint32_t v = lane; v < vpr; v += 32) mx = max(mx, emit(__ldg(xr + v), v, r, yr));
+    }
+    mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+    if (lane == 0) red[warp] = __uint_as_float(mx << 16);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float m = 0.0f;
+        for (int i = 0; i < kWarps; ++i) m = fmaxf(m, red[i]);
+        partials[blockIdx.x] = m;
+    }
+}
+
+}  // namespace
+
+int rmsnorm_grid(int64_t M, int64_t K, int num_sms) {
+    int64_t g = (M + kWarps - 1) / kWarps;
+    (void)K;
+    const int64_t cap = 4LL * num_sms;
+    if (g > cap) g = cap;
+    if (g < 1) g = 1;
+    return static_cast<int>(g);
+}
+
+cudaError_t launch_rmsnorm_amax(const void *x, int64_t M, int64_t K, int64_t ldx, const void *gamma,
+                                float eps, void *y, float *partials, int grid, cudaStream_t s) {
+    return launch_pdl(rmsnorm_amax_kernel, dim3(grid), dim3(kThreads), 0, s,
+                      static_cast<const uint4 *>(x), static_cast<uint32_t>(M),
+                      static_cast<uint32_t>(K / 8), static_cast<uint64_t>(ldx / 8),
+                      static_cast<const uint4 *>(gamma), eps, static_cast<uint4 *>(y), partials);
+}
+
+}  // namespace mq

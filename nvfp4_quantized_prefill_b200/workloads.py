@@ -71,6 +71,13 @@ def weight(N: int, K: int, std: float, seed: int, stream: int,
     return w.to(torch.bfloat16)
 
 
+def rmsnorm_gain(K: int, seed: int, stream: int, device: str = "cpu") -> torch.Tensor:
+    """BF16 [K] RMSNorm gain ~ 1 + N(0, 0.1^2) (a trained gain stays near 1)."""
+    g = _gen(seed, stream, device)
+    v = torch.randn(K, generator=g, dtype=torch.float32, device=device)
+    return (1.0 + 0.1 * v).to(torch.bfloat16)
+
+
 @dataclasses.dataclass(frozen=True)
 class Linear:
     name: str
@@ -91,6 +98,7 @@ class Workload:
     decode_M: Tuple[int, ...]
     swiglu: bool = False        # gate+up -> SwiGLU -> down
     chunks: int = 1             # chunked prefill: M tokens per chunk
+    rmsnorm: bool = False       # the first linear's input = RMSNorm(residual) * gain
 
 
 # Workload table: shapes of the Mix-Quant evaluation's model families at
@@ -109,6 +117,9 @@ WORKLOADS: Dict[str, Workload] = {
         "chunked prefill 131072 tokens in 16384-token chunks", 16384, "student_t3", 3,
         (Linear("o", 4096, 4096, 0.02), Linear("gate_up", 14336, 4096, 0.02)), (1,),
         chunks=8),
+    "llama3_8b_qkv_rmsnorm": Workload(
+        "llama3-8b rmsnorm -> qkv prefill, 8192 tokens", 8192, "channel_gain", 5,
+        (Linear("qkv", 6144, 4096, 0.02),), (1,), rmsnorm=True),
     "llama3_70b_layer": Workload(
         "llama3-70b prefill layer linears, 16384 tokens", 16384, "outlier", 4,
         (Linear("qkv", 10240, 8192, 0.015), Linear("o", 8192, 8192, 0.015),
