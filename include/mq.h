@@ -73,6 +73,14 @@ const char *mq_status_string(mq_status s);
  * check, MQ_ERR_CUDA on a CUDA error, else MQ_OK. */
 mq_status mq_check(cudaStream_t stream);
 
+/* Diagnostic of the failure-detection path (no counterpart on the pages):
+ * queues one tiny kernel that waits, for at most limit_us microseconds
+ * (1 .. 2000000), on a barrier phase that nothing completes, then latches
+ * the same timeout bit the kernels latch when one of their bounded waits runs
+ * out.  The next mq_check on the stream returns MQ_ERR_TIMEOUT (and clears
+ * the bit); the device stays usable.  Never faults or hangs the GPU. */
+mq_status mq_selftest_bounded_wait(uint32_t limit_us, cudaStream_t stream);
+
 /* ---- weights (zingnex "动态精度切换": store weights convertible) ---------- */
 
 /* Builds a weight handle from a BF16 device matrix w_bf16 [N, K] (copied; the

@@ -23,6 +23,7 @@ _P, _I64, _SZ, _I, _U8P = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctyp
 SIGNATURES = [
     ("mq_status_string", ctypes.c_char_p, [_I]),
     ("mq_check", _I, [_P]),
+    ("mq_selftest_bounded_wait", _I, [ctypes.c_uint32, _P]),
     ("mq_weight_pack", _I, [_P, _I64, _I64, _P, ctypes.POINTER(_P)]),
     ("mq_weight_free", _I, [_P]),
     ("mq_weight_views", _I, [_P, ctypes.POINTER(_I64), ctypes.POINTER(_I64), ctypes.POINTER(_P),
@@ -96,6 +97,10 @@ def mq_status_string(code: int) -> str:
 def mq_check(stream=None) -> int:
     """Synchronizes the stream; returns the status (0 or MQ_ERR_*), does not raise."""
     return lib().mq_check(_stream(stream))
+
+
+def mq_selftest_bounded_wait(limit_us: int, stream=None) -> None:
+    _ok("mq_selftest_bounded_wait", lib().mq_selftest_bounded_wait(limit_us, _stream(stream)))
 
 
 def mq_weight_pack(w_bf16, N: int, K: int, stream=None) -> int:

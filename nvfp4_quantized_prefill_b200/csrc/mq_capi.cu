@@ -192,6 +192,47 @@ mq_status mq_check(cudaStream_t stream) {
     return cudaGetLastError() == cudaSuccess ? MQ_OK : MQ_ERR_CUDA;
 }
 
+namespace {
+
+// One CTA, one thread: an mbarrier that expects one arrival nobody makes, a
+// wait on its first phase with the given time limit (%globaltimer), then the
+// same timeout latch the kernels use.  Exits as soon as the limit passes.
+__global__ void selftest_wait_kernel(unsigned long long limit_ns, unsigned *err) {
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(&bar));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(a) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    unsigned long long t0, t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+    for (;;) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(a)
+            : "memory");
+        if (done) return;  // not reachable: nothing arrives
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        if (t - t0 > limit_ns) {
+            atomicOr(err, 1u);  // the timeout bit mq_check reports
+            return;
+        }
+    }
+}
+
+}  // namespace
+
+mq_status mq_selftest_bounded_wait(uint32_t limit_us, cudaStream_t stream) {
+    if (limit_us < 1 || limit_us > 2000000u) return MQ_ERR_INVALID_ARG;
+    DeviceInfo *d = nullptr;
+    mq_status st = device_info(&d);
+    if (st != MQ_OK) return st;
+    selftest_wait_kernel<<<1, 1, 0, stream>>>(static_cast<unsigned long long>(limit_us) * 1000ull,
+                                              d->err);
+    return cudaGetLastError() == cudaSuccess ? MQ_OK : MQ_ERR_CUDA;
+}
+
 size_t mq_sf_bytes(int64_t rows, int64_t K) {
     if (rows < 1 || K < 16) return 0;
     const int64_t rp = (rows + 127) / 128 * 128;

@@ -80,3 +80,19 @@ def test_argument_errors_before_device_work(lib):
     assert L.mq_quantize_nvfp4(16, 4, 64, 64, 16, 16, 16, 16, 0, None, 0, None) == 1
     assert L.mq_weight_free(None) == 0
     assert L.mq_weight_views(None, None, None, None, None, None, None) == 1
+
+
+def test_new_entry_points_reject_bad_arguments_on_the_host(lib):
+    L = lib
+    n = ctypes.c_int()
+    # RMSNorm + amax: null pointers, negative eps, bad K, misaligned x
+    assert L.mq_rmsnorm_amax(None, 16, ctypes.c_float(1e-5), 4, 64, 64, 16, 16, ctypes.byref(n), None) == 1
+    assert L.mq_rmsnorm_amax(16, 16, ctypes.c_float(-1.0), 4, 64, 64, 16, 16, ctypes.byref(n), None) == 1
+    assert L.mq_rmsnorm_amax(16, 16, ctypes.c_float(1e-5), 4, 60, 64, 16, 16, ctypes.byref(n), None) == 2
+    assert L.mq_rmsnorm_amax(24, 16, ctypes.c_float(1e-5), 4, 64, 64, 16, 16, ctypes.byref(n), None) == 3
+    assert L.mq_prefill_linear_rmsnorm_nvfp4(None, None, None, ctypes.c_float(1e-5), 4, None, None,
+                                             None, 0, None) == 1
+    # W4A4 decode and the failure-detection self-test
+    assert L.mq_decode_linear_nvfp4(None, None, 1, None, None, 0, None) == 1
+    assert L.mq_selftest_bounded_wait(0, None) == 1
+    assert L.mq_selftest_bounded_wait(2000001, None) == 1
