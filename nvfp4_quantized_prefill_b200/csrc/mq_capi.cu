@@ -569,7 +569,7 @@ mq_status mq_decode_linear_nvfp4(const mq_weight *w, const void *x_bf16, int64_t
     st = device_info(&d);
     if (st != MQ_OK) return st;
     // up to 8 tokens whose codes fit in shared memory: the kernel quantizes them
-    if (M <= 8 && M * w->K * 9 / 16 <= 160 * 1024)
+    if (M <= 8 && static_cast<size_t>(M * w->K * 9 / 16) <= mq::kDecodeNvf4TokenSmem)
         return cuda_status(mq::launch_decode_nvf4(nullptr, nullptr, nullptr, x_bf16, M, w->codes,
                                                   w->sf, w->s_enc, w->N, w->K, y_bf16,
                                                   w->decode_scratch, d->num_sms, stream));

@@ -196,6 +196,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_nvf4_kernel(
 // partials[group][slice], and the last warp to finish a group (atomic counter,
 // reset by that warp) adds the S slices in order.
 constexpr int kPWarps = 24;
+constexpr size_t kPersistMaxSmem = kDecodeNvf4TokenSmem;
 
 __global__ void __launch_bounds__(kPWarps * 32, 1) decode_nvf4_persist_kernel(
     const __nv_bfloat16 *__restrict__ xb, int M, const uint8_t *__restrict__ wc,
@@ -363,9 +364,12 @@ cudaError_t launch_decode_nvf4(const uint8_t *x_codes, const uint8_t *x_sf, cons
     const int grid = static_cast<int>(groups * S);
     if (x_bf16) {  // M <= 8: tokens quantized in the kernel, persistent warps
         const size_t smem = static_cast<size_t>(M) * static_cast<size_t>(K) * 9u / 16u;  // K/2 + K/16
+        if (smem > kPersistMaxSmem) return cudaErrorInvalidValue;
+        // always the same (largest allowed) value: calls from several host
+        // threads cannot undo each other's setting
         cudaError_t e = cudaFuncSetAttribute(decode_nvf4_persist_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
+                                             static_cast<int>(kPersistMaxSmem));
         if (e != cudaSuccess) return e;
         const int64_t units = groups * S;
         int64_t pgrid = (units + kPWarps - 1) / kPWarps;

@@ -566,16 +566,17 @@ using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, vo
                               CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeFn encode_fn() {
-    static EncodeFn fn = nullptr;
-    if (!fn) {
+    // resolved once; the initialization of a function-local static is
+    // thread-safe
+    static const EncodeFn fn = []() -> EncodeFn {
         void *ptr = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
                 cudaSuccess ||
             q != cudaDriverEntryPointSuccess || !ptr)
             return nullptr;
-        fn = reinterpret_cast<EncodeFn>(ptr);
-    }
+        return reinterpret_cast<EncodeFn>(ptr);
+    }();
     return fn;
 }
 

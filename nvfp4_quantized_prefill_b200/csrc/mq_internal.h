@@ -112,8 +112,13 @@ size_t decode_scratch_bytes(int64_t N, int64_t K, int num_sms);
 cudaError_t launch_decode(const void *x, int64_t M, const void *w, int64_t N, int64_t K,
                           void *y, void *scratch, int num_sms, cudaStream_t s);
 
-// W4A4 decode, weights from the handle's NVFP4 copy.  With x_bf16 set (M <= 8)
-// the kernel quantizes the tokens itself; otherwise x is given quantized
+// Largest M x K x 9 / 16 (bytes of the tokens' codes and scales in shared
+// memory) for which the W4A4 decode quantizes up to 8 tokens itself.
+constexpr size_t kDecodeNvf4TokenSmem = 160 * 1024;
+
+// W4A4 decode, weights from the handle's NVFP4 copy.  With x_bf16 set (M <= 8,
+// M x K x 9 / 16 <= kDecodeNvf4TokenSmem) the kernel quantizes the tokens
+// itself; otherwise x is given quantized
 // (codes, swizzled scales with rows padded to 128, tensor scale).
 cudaError_t launch_decode_nvf4(const uint8_t *x_codes, const uint8_t *x_sf, const float *s_enc_x,
                                const void *x_bf16, int64_t M, const uint8_t *w_codes,

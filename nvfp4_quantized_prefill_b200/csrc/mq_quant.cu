@@ -229,16 +229,17 @@ cudaError_t launch_amax(const void *x, int64_t M, int64_t K, int64_t ldx, float 
 cudaError_t launch_quantize(const void *x, int64_t M, int64_t K, int64_t ldx,
                             const float *partials, int n_partials, uint8_t *codes,
                             uint8_t *sf_swizzled, float *s_enc, int num_sms, cudaStream_t s) {
-    // one resident wave: every CTA pays the scale-table prologue once
-    static int resident = 0;
-    if (resident == 0) {
+    // one resident wave: every CTA pays the scale-table prologue once (the
+    // occupancy is a property of the kernel on sm_100; computed once,
+    // thread-safely)
+    static const int resident = []() {
         int b = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, quantize_kernel, kThreads, 0) !=
                 cudaSuccess ||
             b < 1)
             b = 1;
-        resident = b;
-    }
+        return b;
+    }();
     const int64_t segs = M * ((K + 511) / 512);
     int64_t g = (segs + (kThreads / 32) - 1) / (kThreads / 32);
     const int64_t cap = static_cast<int64_t>(resident) * num_sms;
