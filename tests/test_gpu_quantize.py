@@ -117,3 +117,39 @@ def test_weight_pack_views_bitexact(N, K):
     assert np.array_equal(sf, oracle.sf_swizzle(rsf))
     W.free()
     assert mq.mq_check() == 0
+
+
+def _dynamic_range_matrix(M=256, K=512, seed=4):
+    """Blocks whose magnitudes span 2^-60 .. 2^40: some block scales land in
+    E4M3's subnormal range or underflow to zero relative to the tensor scale,
+    one block holds the tensor maximum, signs and zeros mixed in."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((M, K))
+    exps = rng.integers(-60, 41, size=(M, K // 16))
+    x *= np.repeat(2.0 ** exps, 16, axis=1)
+    x[rng.random((M, K)) < 0.05] = 0.0
+    x[0, :16] = 3.0e12   # a constant block near the top of the range
+    return torch.tensor(x, dtype=torch.float32).to(torch.bfloat16)
+
+
+def test_quantize_dynamic_range_bitexact():
+    x = _dynamic_range_matrix()
+    check_quant(x, "dynamic range")
+    codes, sf, s = gpu_quantize(x.cuda())
+    # blocks far below the maximum quantize to zero scales and zero codes
+    assert (sf == 0).any() and (sf != 0).any()
+
+
+def test_prefill_dynamic_range_within_tolerance():
+    from mqtest import assert_close, oracle_prefill_rows
+    x = _dynamic_range_matrix(128, 512, 5)
+    w = workloads.weight(384, 512, 0.02, 5, 1)
+    W = mq.Weight(w.cuda())
+    y = torch.empty(128, 384, dtype=torch.bfloat16, device="cuda")
+    nb = mq.mq_workspace_bytes(128, 512)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    mq.mq_prefill_linear_nvfp4(W.handle, x.cuda(), 128, y, ws, nb)
+    torch.cuda.synchronize()
+    yr, pr = oracle_prefill_rows(x, w, np.arange(128))
+    assert_close(y.cpu(), yr, pr, "dynamic-range prefill")
+    W.free()
