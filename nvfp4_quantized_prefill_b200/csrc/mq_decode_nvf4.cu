@@ -253,7 +253,9 @@ __global__ void __launch_bounds__(kPWarps * 32, 1) decode_nvf4_persist_kernel(
     const int units = groups * S;
     const int nwarps = gridDim.x * kPWarps;
     const uint2 z2 = make_uint2(0, 0);
-    for (int u = blockIdx.x * kPWarps + warp; u < units; u += nwarps) {
+    // units interleaved across CTAs first, so every SM gets work
+    for (int u = warp * static_cast<int>(gridDim.x) + static_cast<int>(blockIdx.x); u < units;
+         u += nwarps) {
         const int group = u / S, slice = u - group * S;
         const int n0 = group * kRows;
         const int s0 = static_cast<int>(static_cast<int64_t>(steps) * slice / S);
@@ -372,8 +374,7 @@ cudaError_t launch_decode_nvf4(const uint8_t *x_codes, const uint8_t *x_sf, cons
                                              static_cast<int>(kPersistMaxSmem));
         if (e != cudaSuccess) return e;
         const int64_t units = groups * S;
-        int64_t pgrid = (units + kPWarps - 1) / kPWarps;
-        if (pgrid > num_sms) pgrid = num_sms;
+        const int64_t pgrid = units < num_sms ? units : num_sms;   // one CTA per SM
         e = launch_pdl(decode_nvf4_persist_kernel, dim3(static_cast<unsigned>(pgrid)),
                        dim3(kPWarps * 32), smem, s, static_cast<const __nv_bfloat16 *>(x_bf16),
                        static_cast<int>(M), w_codes, w_sf, s_enc_w, static_cast<int>(N),
