@@ -258,13 +258,17 @@ mq_status mq_decode_linear_bf16(const mq_weight *w, const void *x_bf16, int64_t 
  * phases, which the Mix-Quant pages compare their scheme against
  * (gist.science technical summary, section 1 "Problem Statement" and section
  * 4 "Experimental Results"): x is quantized with the prefill recipe (one tensor
- * scale for the call, E4M3 scale per 16, E2M1 codes) into `workspace`, then
+ * scale for the call, E4M3 scale per 16, E2M1 codes), then
  * y[m, n] = bf16( sum_k deq(xq)[m,k] deq(wq)[n,k] / (s_enc_x s_enc_w) ) on the
  * handle's NVFP4 copy, FP32 accumulation -- the same arithmetic as
  * mq_prefill_linear_nvfp4, streaming 0.5625 byte per weight instead of 2.
  * x (device) BF16 [M, K] contiguous, y (device) BF16 [M, N] contiguous; any
- * M >= 1, meant for M <= 8.  workspace (device, 256-byte aligned) of at least
- * mq_workspace_bytes(M, K) bytes.  Shares the handle's split-K scratch with
+ * M >= 1, meant for M <= 16.  Up to 4 tokens, and 9 to 16, whose quantized
+ * form (M K 9/16 bytes) fits in 40 KB run as one tensor-core kernel that
+ * quantizes them in shared memory; up to 8 tokens otherwise as one FP16-MMA
+ * kernel that does the same; else x is quantized into `workspace` first.
+ * workspace (device, 256-byte aligned) of at least mq_workspace_bytes(M, K)
+ * bytes in every case.  Shares the handle's split-K scratch with
  * mq_decode_linear_bf16: decode calls on one handle must not overlap on the
  * GPU. */
 mq_status mq_decode_linear_nvfp4(const mq_weight *w, const void *x_bf16, int64_t M, void *y_bf16,

@@ -568,8 +568,17 @@ mq_status mq_decode_linear_nvfp4(const mq_weight *w, const void *x_bf16, int64_t
     DeviceInfo *d = nullptr;
     st = device_info(&d);
     if (st != MQ_OK) return st;
-    // up to 8 tokens whose codes fit in shared memory: the kernel quantizes them
-    if (M <= 8 && static_cast<size_t>(M * w->K * 9 / 16) <= mq::kDecodeNvf4TokenSmem)
+    const size_t tok_bytes = static_cast<size_t>(M) * static_cast<size_t>(w->K) * 9u / 16u;
+    const bool tc_fits = M <= mq::kDecodeTcTokens && tok_bytes + 15u <= mq::kDecodeTcTokenSmem;
+    // the tensor-core kernel (quantizes the tokens itself, one pass over the
+    // weight) for up to 4 tokens; for 5 to 8, where every CTA quantizing all
+    // tokens costs it more than the FP16 dequantization costs the FP16-MMA
+    // kernel, that one; the tensor-core kernel again for 9 to 16
+    if (tc_fits && (M <= 4 || M > 8))
+        return cuda_status(mq::launch_decode_nvf4_tc(w->tmap, w->sf, w->s_enc, w->N, w->K, x_bf16,
+                                                     M, y_bf16, w->decode_scratch, d->err,
+                                                     d->num_sms, stream));
+    if (M <= 8 && tok_bytes <= mq::kDecodeNvf4TokenSmem)
         return cuda_status(mq::launch_decode_nvf4(nullptr, nullptr, nullptr, x_bf16, M, w->codes,
                                                   w->sf, w->s_enc, w->N, w->K, y_bf16,
                                                   w->decode_scratch, d->num_sms, stream));

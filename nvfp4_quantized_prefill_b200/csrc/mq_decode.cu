@@ -13,11 +13,16 @@
 // up to 8 X rows as N.  Both fragments take the same K permutation (the 8
 // elements a thread loads), so no shuffles or staging are needed; for 8 tokens
 // the tensor core does the 8 FMAs per weight element that would otherwise
-// load the FP32 pipes.  K is split into S slices so that there are enough
-// units to balance the SMs; the last CTA of a row group to finish (an atomic
+// load the FP32 pipes.  A CTA's unit is 16 whole consecutive rows when there
+// are enough row groups (one contiguous block of W).  The weight loads of
+// eight steps are issued together, before their MMAs (8 KB in flight per
+// warp).  With fewer row groups than SMs, K is split into S slices so that
+// every SM gets two to three CTAs, all resident at once (the register budget
+// allows three per SM); the last CTA of a row group to finish (an atomic
 // counter, reset by that CTA) adds the S partial sums in slice order --
-// deterministically -- and writes BF16.  Scratch (per weight): one counter per
-// row group first, then the partial sums.
+// deterministically -- and writes BF16.
+// Scratch (per weight): one counter per row group first, then the partial
+// sums.
 #include <cuda_bf16.h>
 
 #include "mq_internal.h"
@@ -29,6 +34,17 @@ namespace {
 constexpr int kWarps = 8;
 constexpr int kRows = 16;
 constexpr int kUnroll = 8;
+constexpr int kCtasPerSm = 3;   // register budget: the grid of a split K is resident at once
+
+// W is streamed once: the loads are issued as written (all of a batch before
+// its MMAs), not sunk towards their use.
+__device__ __forceinline__ uint4 ld_w(const uint4 *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
 
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                                uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -39,7 +55,7 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__global__ void __launch_bounds__(kWarps * 32) decode_kernel(const uint4 *__restrict__ x, int M,
+__global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_kernel(const uint4 *__restrict__ x, int M,
                                                              const uint4 *__restrict__ w, int N,
                                                              int K, int S,
                                                              __nv_bfloat16 *__restrict__ y,
@@ -59,20 +75,21 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(const uint4 *__rest
     const int sl1 = static_cast<int>(static_cast<int64_t>(steps) * (slice + 1) / S);
     const int s0 = sl0 + (sl1 - sl0) * warp / kWarps;
     const int s1 = sl0 + (sl1 - sl0) * (warp + 1) / kWarps;
-    const bool ra = n0 + g < N, rb = n0 + g + 8 < N, rx = g < M;
-    const uint4 *wa = w + static_cast<int64_t>(ra ? n0 + g : 0) * vpr + t4;
-    const uint4 *wb = w + static_cast<int64_t>(rb ? n0 + g + 8 : 0) * vpr + t4;
-    const uint4 *xr = x + static_cast<int64_t>(rx ? g : 0) * vpr + t4;
-    const uint4 z = make_uint4(0, 0, 0, 0);
+    // rows past N read row N - 1 and tokens past M read token 0: those
+    // accumulator entries are never written out
+    const int ra = n0 + g < N ? n0 + g : N - 1, rb = n0 + g + 8 < N ? n0 + g + 8 : N - 1;
+    const uint4 *wa = w + static_cast<int64_t>(ra) * vpr + t4;
+    const uint4 *wb = w + static_cast<int64_t>(rb) * vpr + t4;
+    const uint4 *xr = x + static_cast<int64_t>(g < M ? g : 0) * vpr + t4;
     float c[4] = {0.f, 0.f, 0.f, 0.f};
     int s = s0;
     for (; s + kUnroll <= s1; s += kUnroll) {
         uint4 va[kUnroll], vb[kUnroll], vx[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            va[u] = ra ? __ldg(wa + (s + u) * 4) : z;
-            vb[u] = rb ? __ldg(wb + (s + u) * 4) : z;
-            vx[u] = rx ? __ldg(xr + (s + u) * 4) : z;
+            va[u] = ld_w(wa + (s + u) * 4);
+            vb[u] = ld_w(wb + (s + u) * 4);
+            vx[u] = __ldg(xr + (s + u) * 4);
         }
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
@@ -81,9 +98,9 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(const uint4 *__rest
         }
     }
     for (; s < s1; ++s) {
-        const uint4 va = ra ? __ldg(wa + s * 4) : z;
-        const uint4 vb = rb ? __ldg(wb + s * 4) : z;
-        const uint4 vx = rx ? __ldg(xr + s * 4) : z;
+        const uint4 va = ld_w(wa + s * 4);
+        const uint4 vb = ld_w(wb + s * 4);
+        const uint4 vx = __ldg(xr + s * 4);
         mma_bf16_16816(c, va.x, vb.x, va.y, vb.y, vx.x, vx.y);
         mma_bf16_16816(c, va.z, vb.z, va.w, vb.w, vx.z, vx.w);
     }
@@ -122,7 +139,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(const uint4 *__rest
 
 int decode_slices(int64_t N, int64_t K, int num_sms) {
     const int64_t groups = (N + kRows - 1) / kRows;
-    if (groups >= 2LL * num_sms) return 1;               // enough row groups to balance
+    if (groups >= num_sms) return 1;   // whole rows: no partial sums, one block of W a CTA
     int64_t S = (2LL * num_sms + groups - 1) / groups;   // >= 2 CTAs per SM
     const int64_t max_s = K / 512 > 0 ? K / 512 : 1;     // keep >= 16 steps per slice
     if (S > max_s) S = max_s;
@@ -140,9 +157,11 @@ size_t decode_scratch_bytes(int64_t N, int64_t K, int num_sms) {
     int S = decode_slices(N, K, num_sms);
     const int S4 = decode_nvf4_slices(N, K, num_sms);
     if (S4 > S) S = S4;
-    if (S == 1) return 0;
     const int64_t groups = (N + kRows - 1) / kRows;
-    return decode_counter_bytes(N) + static_cast<size_t>(groups) * S * 128 * sizeof(float);
+    size_t floats = static_cast<size_t>(groups) * S * 128;
+    const size_t tc = decode_tc_partial_floats(N, K, num_sms);
+    if (tc > floats) floats = tc;
+    return decode_counter_bytes(N) + floats * sizeof(float);
 }
 
 cudaError_t launch_decode(const void *x, int64_t M, const void *w, int64_t N, int64_t K, void *y,

@@ -99,11 +99,12 @@ bool encode_sf_tmap(CUtensorMap *map, const void *sf, int64_t rows, int64_t K);
 
 // ---- decode (mq_decode.cu: BF16; mq_decode_nvf4.cu: NVFP4 W4A4) ----------------
 
-// Number of K slices the BF16 / NVFP4 decode splits an [N, K] weight into,
-// and the bytes of per-weight scratch they need (0 when both use S = 1): one
-// counter per 16-row group (decode_counter_bytes, at the start; the counters
-// must start at zero and are left at zero by every launch), then S x 128 FP32
-// partial sums per group for the larger S.
+// Number of K slices the BF16 / NVFP4 (FP16-MMA) decode splits an [N, K]
+// weight into, and the bytes of per-weight decode scratch: one counter per
+// 16-row group (decode_counter_bytes, at the start; the counters must start
+// at zero and are left at zero by every launch), then the FP32 partial sums
+// of whichever decode kernel needs the most (S x 128 per 16-row group, or the
+// tensor-core decode's decode_tc_partial_floats).
 int decode_slices(int64_t N, int64_t K, int num_sms);
 int decode_nvf4_slices(int64_t N, int64_t K, int num_sms);
 size_t decode_counter_bytes(int64_t N);
@@ -124,5 +125,20 @@ cudaError_t launch_decode_nvf4(const uint8_t *x_codes, const uint8_t *x_sf, cons
                                const void *x_bf16, int64_t M, const uint8_t *w_codes,
                                const uint8_t *w_sf, const float *s_enc_w, int64_t N, int64_t K,
                                void *y, void *scratch, int num_sms, cudaStream_t s);
+
+// W4A4 decode on the tcgen05 tensor cores (mq_decode_tc.cu) for up to
+// kDecodeTcTokens BF16 tokens x [M, K] whose NVFP4 form (M K 9 / 16 bytes)
+// fits in kDecodeTcTokenSmem; the kernel quantizes them itself.  tmap_w is
+// the weight codes' tensor map (encode_codes_tmap).  The weight is read
+// before the wait on the preceding kernel: no kernel may write it just before
+// (packing ends with a memory set).  decode_tc_partial_floats is the FP32
+// partial-sum space it needs after the per-weight counters.
+constexpr int64_t kDecodeTcTokens = 16;
+constexpr size_t kDecodeTcTokenSmem = 40 * 1024;
+size_t decode_tc_partial_floats(int64_t N, int64_t K, int num_sms);
+cudaError_t launch_decode_nvf4_tc(const CUtensorMap &tmap_w, const uint8_t *w_sf,
+                                  const float *s_enc_w, int64_t N, int64_t K, const void *x_bf16,
+                                  int64_t M, void *y, void *scratch, unsigned *err, int num_sms,
+                                  cudaStream_t s);
 
 }  // namespace mq

@@ -151,12 +151,17 @@ __device__ __forceinline__ float nvfp4_tensor_scale(float amax) {
 }
 
 // ftab[b] = s_enc / dec(b) (0 for dec(b) = 0) for the 128 non-negative E4M3
-// bytes; threads 0..127 of the block each write one entry.
-__device__ __forceinline__ void nvfp4_scale_table(float s_enc, float *ftab) {
-    if (threadIdx.x < 128) {
-        const float dec = e4m3_to_float(threadIdx.x);
-        ftab[threadIdx.x] = dec == 0.0f ? 0.0f : __fdiv_rn(s_enc, dec);
+// bytes, written by threads tid = 0 .. nthreads - 1 (by default threads
+// 0..127 of the block, one entry each).
+__device__ __forceinline__ void nvfp4_scale_table(float s_enc, float *ftab, uint32_t tid,
+                                                  uint32_t nthreads) {
+    for (uint32_t b = tid; b < 128u; b += nthreads) {
+        const float dec = e4m3_to_float(b);
+        ftab[b] = dec == 0.0f ? 0.0f : __fdiv_rn(s_enc, dec);
     }
+}
+__device__ __forceinline__ void nvfp4_scale_table(float s_enc, float *ftab) {
+    if (threadIdx.x < 128) nvfp4_scale_table(s_enc, ftab, threadIdx.x, 128u);
 }
 
 }  // namespace mq

@@ -244,8 +244,12 @@ cudaError_t launch_quantize(const void *x, int64_t M, int64_t K, int64_t ldx,
     int64_t g = (segs + (kThreads / 32) - 1) / (kThreads / 32);
     const int64_t cap = static_cast<int64_t>(resident) * num_sms;
     if (g > cap) g = cap;
-    if (g < 1) g = 1;
     const int64_t Mpad = (M + 127) / 128 * 128;
+    // enough CTAs for the padding rows' scale words too (about 8 per thread):
+    // a handful of tokens would otherwise leave ~8000 words to one CTA
+    const int64_t gpad = ((Mpad - M) * (K / 64) + kThreads * 8 - 1) / (kThreads * 8);
+    if (g < gpad) g = gpad < cap ? gpad : cap;
+    if (g < 1) g = 1;
     return launch_pdl(quantize_kernel, dim3(static_cast<unsigned>(g)), dim3(kThreads), 0, s,
                       static_cast<const uint4 *>(x), static_cast<uint32_t>(M),
                       static_cast<uint32_t>(K), static_cast<uint64_t>(ldx / 8), partials,

@@ -26,11 +26,15 @@ def gpu_decode_nvfp4(x_cpu, W):
     return y.cpu()
 
 
-# (M, N, K): one token; 8 tokens with ragged N and a partial last 256-K step;
-# N < 16; more than 8 tokens (two launches); N = 1; split-K (few row groups,
-# long K); a long-K 8-token case.
+# (M, N, K): one token; 8 tokens with ragged N and a partial last 256-K step
+# (FP16-MMA kernel); N < 16; 13 and 16 tokens (the tensor-core kernel's limit)
+# and 17 (quantize kernels + FP16-MMA kernel, two launches); N = 1; few weight
+# rows with a long K (tiles split across many CTAs); a long-K 8-token case;
+# a partial last K step of three scale blocks; the Llama-3-8B QKV shape.
+# Tensor-core kernel: M <= 4 or 9..16 with M K 9/16 <= 40 KB.
 SHAPES = [(1, 256, 256), (8, 300, 320), (3, 17, 64), (13, 1024, 4096), (1, 1, 128),
-          (2, 64, 8192), (1, 16, 16384), (8, 4096, 14336), (5, 100, 448)]
+          (2, 64, 8192), (1, 16, 16384), (8, 4096, 14336), (5, 100, 448), (16, 520, 1024),
+          (17, 200, 512), (1, 6144, 4096), (4, 1000, 2048)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES)

@@ -27,7 +27,7 @@ def gpu_decode(x_cpu, W):
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 256, 256), (8, 300, 320), (3, 17, 64), (13, 1024, 4096),
-                                   (1, 1, 128), (8, 4096, 14336)])
+                                   (1, 1, 128), (8, 4096, 14336), (2, 6150, 4096), (1, 33, 8192)])
 def test_decode_small(M, N, K):
     x = workloads.activation("outlier", M, K, 2, M)
     w = workloads.weight(N, K, 0.02, 2, N)
@@ -37,6 +37,28 @@ def test_decode_small(M, N, K):
     assert_close(y, yr, pr, f"decode {M}x{N}x{K}")
     W.free()
     assert mq.mq_check() == 0
+
+
+def test_decode_deterministic_and_reusable():
+    """Groups shared by several warps are summed in a fixed order: repeated
+    calls give the same bits, and the per-weight counters are left ready for
+    calls with another M on the same handle."""
+    N, K = 6144, 4096
+    w = workloads.weight(N, K, 0.02, 3, 0)
+    W = mq.Weight(w.cuda())
+    x = workloads.activation("outlier", 8, K, 3, 1)
+    first = gpu_decode(x, W)
+    for M in (1, 8, 3, 8):
+        y = gpu_decode(x[:M], W)
+        assert torch.equal(u16_t(y), u16_t(first[:M])), M
+    yr, pr = oracle.decode_linear(x, w)
+    assert_close(first, yr, pr, "decode 8x6144x4096")
+    W.free()
+    assert mq.mq_check() == 0
+
+
+def u16_t(y):
+    return y.view(torch.int16)
 
 
 def test_decode_phase_switch_llama8b_mlp_weights():
