@@ -97,6 +97,27 @@ def test_quantize_strided_rows_and_external_amax():
     assert mq.mq_check() == 0
 
 
+def test_quantize_amax_inside_strided_and_workspace_reuse():
+    """Amax taken inside mq_quantize_nvfp4 (partial maxima in the workspace):
+    strided rows, and a workspace reused across calls -- the second call (a
+    much smaller amax) must not see the first call's partial maxima."""
+    ws = torch.empty(mq.MQ_AMAX_PARTIALS_MAX, dtype=torch.float32, device="cuda")
+    for M, K, ld, gain in ((3000, 4096, 4160, 30.0), (3000, 4096, 4160, 0.01), (17, 448, 448, 1.0)):
+        full = (workloads.activation("outlier", M, ld, 4, 1).float() * gain).to(torch.bfloat16)
+        x_cpu = full[:, :K].contiguous()
+        codes = torch.empty(M, K // 2, dtype=torch.uint8, device="cuda")
+        sf = torch.empty(mq.mq_sf_bytes(M, K), dtype=torch.uint8, device="cuda")
+        s = torch.empty(1, dtype=torch.float32, device="cuda")
+        mq.mq_quantize_nvfp4(full.cuda(), M, K, ld, codes, sf, s, workspace=ws,
+                             ws_bytes=ws.numel() * 4)
+        torch.cuda.synchronize()
+        rc, rsf, rs, _ = oracle.quantize_tensor(x_cpu)
+        assert float(s.item()) == rs, (M, K, gain)
+        assert np.array_equal(codes.cpu().numpy(), rc), (M, K, gain)
+        assert np.array_equal(sf.cpu().numpy(), oracle.sf_swizzle(rsf)), (M, K, gain)
+    assert mq.mq_check() == 0
+
+
 @pytest.mark.parametrize("N,K", [(520, 320), (256, 256), (6144, 4096)])
 def test_weight_pack_views_bitexact(N, K):
     w = workloads.weight(N, K, 0.02, 5, N)
