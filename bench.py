@@ -472,12 +472,19 @@ def run_gpu(args, wl, world, rank):
         return statistics.mean(ts)
 
     decode_timing = "cuda-graph replay"
+    op_device_us = {}
     try:
         g_flush, g_dec, g_dec4 = capture([]), capture(P.dec), capture(P.dec4)
         t_flush = replay_ms(g_flush)
         t_dec_iso = (replay_ms(g_dec) - t_flush) / R
         t_dec4 = (replay_ms(g_dec4) - t_flush) / R
         del g_flush, g_dec, g_dec4
+        # every prefill launch alone on a cold L2, same method (device time;
+        # inside the step a quantize finds X partly in L2 after its amax)
+        for name, _, f in P.ops:
+            g = capture([f])
+            op_device_us[name] = round((replay_ms(g) - t_flush) / R * 1e3, 2)
+            del g
     except Exception as e:  # report, do not hide
         decode_timing = f"eager (graph capture failed: {type(e).__name__})"
         torch.cuda.synchronize()
@@ -703,6 +710,11 @@ def run_gpu(args, wl, world, rank):
                        "the flush alone; NVFP4 = W4A4, tokens quantized inside the kernel; "
                        "GB/s over the weight bytes (2 or 0.5625 B/param) + x + y",
         "decode_timing": decode_timing,
+        "op_device_us": op_device_us,
+        "op_device_note": "each prefill launch alone after an L2 flush, device time from "
+                          "CUDA-graph replays (16 x (flush, launch) minus 16 flushes); "
+                          "per_launch_ms, from events between launches, also holds the "
+                          "launch gaps",
         "graph_prefill_ms": round(graph_ms, 4) if isinstance(graph_ms, float) else graph_ms,
         "tokens_per_s": round(world * wl.M * max(1, wl.chunks) / (t_prefill_max * 1e-3), 1),
         "fp4_peak_frac": round(value / fp4_peak, 4),
