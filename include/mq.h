@@ -119,6 +119,15 @@ size_t mq_sf_bytes(int64_t rows, int64_t K);
 mq_status mq_tensor_amax(const void *x_bf16, int64_t M, int64_t K, int64_t ldx,
                          float *amax_partials, int *n_partials, cudaStream_t stream);
 
+/* amax_out[0] = max(amax_partials[0 .. n_partials)) on the device (one
+ * kernel): the tensor amax as one float, for instance to take its max over
+ * the token shards of a batch split across GPUs, so that every shard is
+ * quantized with the scale of the whole batch (then pass amax_out with
+ * n_partials = 1 to mq_quantize_nvfp4).  Both pointers device, 4-byte
+ * aligned; 1 <= n_partials <= MQ_AMAX_PARTIALS_MAX. */
+mq_status mq_amax_combine(const float *amax_partials, int n_partials, float *amax_out,
+                          cudaStream_t stream);
+
 /* NVFP4-quantizes a BF16 device matrix x [M, K] (ldx as above, K % 64 == 0).
  *   amax_partials / n_partials: device array of partial maxima whose max is
  *     the tensor amax (from mq_tensor_amax or a fused epilogue); pass NULL to

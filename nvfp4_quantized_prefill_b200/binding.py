@@ -30,6 +30,7 @@ SIGNATURES = [
                              ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P)]),
     ("mq_sf_bytes", _SZ, [_I64, _I64]),
     ("mq_tensor_amax", _I, [_P, _I64, _I64, _I64, _P, ctypes.POINTER(_I), _P]),
+    ("mq_amax_combine", _I, [_P, _I, _P, _P]),
     ("mq_quantize_nvfp4", _I, [_P, _I64, _I64, _I64, _U8P, _U8P, _P, _P, _I, _P, _SZ, _P]),
     ("mq_gemm_nvfp4", _I, [_U8P, _U8P, _P, _I64, _P, _P, _I64, _P]),
     ("mq_gemm_nvfp4_swiglu", _I, [_U8P, _U8P, _P, _I64, _P, _P, _P, ctypes.POINTER(_I), _P]),
@@ -140,6 +141,11 @@ def mq_tensor_amax(x, M: int, K: int, ldx: int, amax_partials, stream=None) -> i
     _ok("mq_tensor_amax", lib().mq_tensor_amax(_ptr(x), M, K, ldx, _ptr(amax_partials),
                                                ctypes.byref(n), _stream(stream)))
     return n.value
+
+
+def mq_amax_combine(amax_partials, n_partials: int, amax_out, stream=None) -> None:
+    _ok("mq_amax_combine", lib().mq_amax_combine(_ptr(amax_partials), n_partials, _ptr(amax_out),
+                                                 _stream(stream)))
 
 
 def mq_quantize_nvfp4(x, M: int, K: int, ldx: int, codes, sf_swizzled, s_enc, amax_partials=None,

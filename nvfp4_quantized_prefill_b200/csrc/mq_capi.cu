@@ -337,6 +337,18 @@ mq_status mq_tensor_amax(const void *x_bf16, int64_t M, int64_t K, int64_t ldx,
     return cuda_status(mq::launch_amax(x_bf16, M, K, ldx, amax_partials, g, stream));
 }
 
+mq_status mq_amax_combine(const float *amax_partials, int n_partials, float *amax_out,
+                          cudaStream_t stream) {
+    if (!amax_partials || !amax_out) return MQ_ERR_INVALID_ARG;
+    if (n_partials < 1 || n_partials > MQ_AMAX_PARTIALS_MAX) return MQ_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(amax_partials) & 3u) || (reinterpret_cast<uintptr_t>(amax_out) & 3u))
+        return MQ_ERR_ALIGNMENT;
+    DeviceInfo *d = nullptr;
+    mq_status st = device_info(&d);
+    if (st != MQ_OK) return st;
+    return cuda_status(mq::launch_amax_combine(amax_partials, n_partials, amax_out, stream));
+}
+
 mq_status mq_quantize_nvfp4(const void *x_bf16, int64_t M, int64_t K, int64_t ldx,
                             uint8_t *codes, uint8_t *sf_swizzled, float *s_enc_dev,
                             const float *amax_partials, int n_partials, void *workspace,

@@ -54,6 +54,9 @@ int amax_grid(int64_t M, int64_t K, int num_sms);
 cudaError_t launch_amax(const void *x, int64_t M, int64_t K, int64_t ldx, float *partials,
                         int grid, cudaStream_t s);
 
+// out[0] = max(partials[0..n)) (one CTA).
+cudaError_t launch_amax_combine(const float *partials, int n, float *out, cudaStream_t s);
+
 // NVFP4 quantization with the tensor amax = max(partials[0..n_partials)).
 cudaError_t launch_quantize(const void *x, int64_t M, int64_t K, int64_t ldx,
                             const float *partials, int n_partials, uint8_t *codes,

@@ -208,6 +208,19 @@ __global__ void __launch_bounds__(kThreads, kQuantBlocksPerSm) quantize_kernel(
     }
 }
 
+// max(partials[0 .. n)) into out[0]: the tensor amax as one float, e.g. to be
+// combined across token shards (max is exact and order-free).
+__global__ void __launch_bounds__(kThreads) amax_combine_kernel(const float *__restrict__ partials,
+                                                                int n, float *__restrict__ out) {
+    __shared__ float red[kThreads / 32];
+    griddep_wait();
+    griddep_launch_dependents();
+    float m = 0.0f;
+    for (int i = threadIdx.x; i < n; i += kThreads) m = fmaxf(m, partials[i]);
+    m = block_max(m, red);
+    if (threadIdx.x == 0) out[0] = m;
+}
+
 }  // namespace
 
 int amax_grid(int64_t M, int64_t K, int num_sms) {
@@ -255,6 +268,10 @@ cudaError_t launch_quantize(const void *x, int64_t M, int64_t K, int64_t ldx,
                       static_cast<uint32_t>(K), static_cast<uint64_t>(ldx / 8), partials,
                       n_partials, reinterpret_cast<uint2 *>(codes), sf_swizzled, s_enc,
                       static_cast<uint32_t>(Mpad));
+}
+
+cudaError_t launch_amax_combine(const float *partials, int n, float *out, cudaStream_t s) {
+    return launch_pdl(amax_combine_kernel, dim3(1), dim3(kThreads), 0, s, partials, n, out);
 }
 
 }  // namespace mq

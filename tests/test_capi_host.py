@@ -96,3 +96,8 @@ def test_new_entry_points_reject_bad_arguments_on_the_host(lib):
     assert L.mq_decode_linear_nvfp4(None, None, 1, None, None, 0, None) == 1
     assert L.mq_selftest_bounded_wait(0, None) == 1
     assert L.mq_selftest_bounded_wait(2000001, None) == 1
+    # amax combine (token sharding): null pointers, count out of range, misalignment
+    assert L.mq_amax_combine(None, 4, 16, None) == 1
+    assert L.mq_amax_combine(16, 0, 16, None) == 1
+    assert L.mq_amax_combine(16, 4097, 16, None) == 1
+    assert L.mq_amax_combine(18, 4, 16, None) == 3
