@@ -21,17 +21,23 @@ def _built():
 
 
 def check_rows(y_gpu_u16: np.ndarray, y_ref_u16: np.ndarray, what: str):
-    """At most one BF16 step apart (the binary32 vs binary64 reciprocal root),
-    and identical almost everywhere."""
+    """Identical almost everywhere, and never more than two BF16 steps apart.
+    The binary32 reciprocal root r can differ from the binary64 one by an ulp,
+    which moves t = bf16(x r) by at most one step (|t| 2^-7); y = bf16(g t)
+    then moves by |g| |t| 2^-7 ~ |y| 2^-7 plus its own rounding step, hence
+    two steps of |y| 2^-7."""
     yg = torch.from_numpy(y_gpu_u16.view(np.int16)).view(torch.bfloat16).double()
     yr = torch.from_numpy(y_ref_u16.view(np.int16)).view(torch.bfloat16).double()
     step = torch.where(yr == 0, torch.full_like(yr, 2.0 ** -133), yr.abs() * 2.0 ** -7)
-    assert ((yg - yr).abs() <= step * 1.0001).all(), what
+    assert ((yg - yr).abs() <= 2.0 * step * 1.0001).all(), what
     assert (y_gpu_u16 == y_ref_u16).mean() > 0.999, what
 
 
+# K <= 4096 and K <= 8192: the CTA-per-row kernel's two forms; K = 16384: the
+# warp-per-row kernel
 @pytest.mark.parametrize("M,K,ldx", [(1, 64, 64), (37, 320, 328), (300, 4096, 4096),
-                                     (8, 8192, 8192), (5, 8, 8)])
+                                     (8, 8192, 8192), (5, 8, 8), (1000, 2048, 2056),
+                                     (20, 16384, 16384), (700, 6144, 6144)])
 def test_rmsnorm_amax(M, K, ldx):
     x = workloads.activation("channel_gain", M, ldx, 21, M)
     g = workloads.rmsnorm_gain(K, 21, 1)
