@@ -341,7 +341,8 @@ mq_status mq_amax_combine(const float *amax_partials, int n_partials, float *ama
                           cudaStream_t stream) {
     if (!amax_partials || !amax_out) return MQ_ERR_INVALID_ARG;
     if (n_partials < 1 || n_partials > MQ_AMAX_PARTIALS_MAX) return MQ_ERR_INVALID_ARG;
-    if ((reinterpret_cast<uintptr_t>(amax_partials) & 3u) || (reinterpret_cast<uintptr_t>(amax_out) & 3u))
+    if ((reinterpret_cast<uintptr_t>(amax_partials) & 3u) ||
+        (reinterpret_cast<uintptr_t>(amax_out) & 3u))
         return MQ_ERR_ALIGNMENT;
     DeviceInfo *d = nullptr;
     mq_status st = device_info(&d);

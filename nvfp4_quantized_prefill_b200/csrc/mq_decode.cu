@@ -55,12 +55,10 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) decode_kernel(const uint4 *__restrict__ x, int M,
-                                                             const uint4 *__restrict__ w, int N,
-                                                             int K, int S,
-                                                             __nv_bfloat16 *__restrict__ y,
-                                                             float *__restrict__ partials,
-                                                             unsigned *__restrict__ counters) {
+__global__ void __launch_bounds__(kWarps * 32, kCtasPerSm)
+    decode_kernel(const uint4 *__restrict__ x, int M, const uint4 *__restrict__ w, int N, int K,
+                  int S, __nv_bfloat16 *__restrict__ y, float *__restrict__ partials,
+                  unsigned *__restrict__ counters) {
     __shared__ float part[kWarps][128];
     __shared__ int last;
     griddep_wait();

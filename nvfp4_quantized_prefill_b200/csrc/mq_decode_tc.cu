@@ -13,12 +13,16 @@
 // The op streams the NVFP4 weight once (0.5625 byte per parameter); the
 // tensor core does the E2M1 decoding and the block scaling that an FP16 MMA
 // path spends most of its instructions on.  The tokens' NVFP4 form must fit
-// in shared memory (M K 9 / 16 <= kDecodeTcTokenSmem).  The weight is the MMA's A operand
-// (M = 128 weight rows) and the tokens its B operand (N = 16; token rows past
-// M stay zero), K = 64 per instruction with one UE4M3 scale per 16 K.  Work
-// unit: one 128-row weight tile x one 256-wide K stage; the flattened
-// (tile, stage) sequence is split into equal contiguous ranges, one per CTA
-// (one CTA per SM), so every SM streams the same bytes.
+// in shared memory (M K 9 / 16 <= kDecodeTcTokenSmem).  The weight is the
+// MMA's A operand (M = 128 weight rows) and the tokens its B operand (N = 16;
+// token rows past M stay zero), K = 64 per instruction with one UE4M3 scale
+// per 16 K.  Work unit: one 128-row weight tile x one 256-wide K stage; the
+// flattened (tile, stage) sequence is split into equal contiguous ranges, one
+// per CTA (one CTA per SM), so every SM streams the same bytes.  Each CTA's
+// few stages are short next to its fixed path (set-up, the first TMA round
+// trip, the token quantization, the accumulator hand-off and the cross-CTA
+// reduction), so the library uses it for up to 4 tokens and for 9 to 16; for
+// 5 to 8 the FP16-MMA kernel is faster.
 //
 // CTA roles (9 warps):
 //   warp 0     TMA producer: weight codes [128 x 128 B] (128-byte swizzle)
