@@ -64,7 +64,8 @@ def test_decode_nvfp4_phase_switch_llama8b_qkv():
 
 def test_decode_paths_share_scratch():
     """BF16 and NVFP4 decode on one split-K handle, alternating: each leaves
-    the shared counters at zero for the other."""
+    the shared counters at zero for the other, and every round gives the same
+    bits (the split-K partial sums are added in a fixed order)."""
     import oracle
     M, N, K = 2, 48, 8192
     x = workloads.activation("student_t3", M, K, 8, 0)
@@ -72,12 +73,17 @@ def test_decode_paths_share_scratch():
     W = mq.Weight(w.cuda())
     yr4, pr4 = oracle_prefill_rows(x, w, np.arange(M))
     yr16, pr16 = oracle.decode_linear(x, w)
+    first = None
     for it in range(3):
         y16 = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
         mq.mq_decode_linear_bf16(W.handle, x.cuda(), M, y16)
         y4 = gpu_decode_nvfp4(x, W)
         assert_close(y16.cpu(), yr16, pr16, f"bf16 decode round {it}")
         assert_close(y4, yr4, pr4, f"nvfp4 decode round {it}")
+        if first is None:
+            first = (y16.cpu(), y4)
+        assert torch.equal(y16.cpu().view(torch.int16), first[0].view(torch.int16)), it
+        assert torch.equal(y4.view(torch.int16), first[1].view(torch.int16)), it
     W.free()
     assert mq.mq_check() == 0
 
