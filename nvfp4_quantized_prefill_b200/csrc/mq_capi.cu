@@ -283,14 +283,19 @@ mq_status mq_weight_pack(const void *w_bf16, int64_t N, int64_t K, cudaStream_t 
     w->s_enc = reinterpret_cast<float *>(w->sf + b_sf + b_part);
     w->decode_scratch = b_dec ? static_cast<void *>(w->sf + b_sf + b_part + 256) : nullptr;
     st = MQ_OK;
-    if (b_dec && cudaMemsetAsync(w->decode_scratch, 0, b_dec, stream) != cudaSuccess)
-        st = MQ_ERR_CUDA;
-    if (st == MQ_OK && cudaMemcpyAsync(w->bf16, w_bf16, static_cast<size_t>(N) * K * 2,
-                                       cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
+    if (cudaMemcpyAsync(w->bf16, w_bf16, static_cast<size_t>(N) * K * 2,
+                        cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
         st = MQ_ERR_CUDA;
     if (st == MQ_OK)
         st = quantize_impl(d, w->bf16, N, K, K, w->codes, w->sf, w->s_enc, nullptr, 0, w->partials,
                            stream);
+    // Last on the stream, and not a kernel: the tensor-core W4A4 decode reads
+    // the weight before its wait on the preceding kernel (programmatic
+    // dependent launch), so it must never directly follow the kernel that
+    // writes the codes; a memory set in between orders it fully.  (b_dec is
+    // never 0: the counters alone take 256 bytes.)
+    if (st == MQ_OK && cudaMemsetAsync(w->decode_scratch, 0, b_dec, stream) != cudaSuccess)
+        st = MQ_ERR_CUDA;
     if (st == MQ_OK && (!mq::encode_codes_tmap(&w->tmap, w->codes, N, K) ||
                         !mq::encode_sf_tmap(&w->tmap_sf, w->sf, N, K)))
         st = MQ_ERR_CUDA;

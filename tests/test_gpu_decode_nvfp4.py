@@ -62,6 +62,28 @@ def test_decode_nvfp4_phase_switch_llama8b_qkv():
     W.free()
 
 
+def test_decode_nvfp4_right_after_packing():
+    """No operation between packing the weight and the decode: the
+    tensor-core kernel streams the weight before waiting on the kernel before
+    it, and packing ends with a memory set, so that kernel is never the one
+    that writes the codes."""
+    M, N, K = 1, 6144, 4096
+    x = workloads.activation("outlier", M, K, 12, 0)
+    w = workloads.weight(N, K, 0.02, 12, 1)
+    xd, wd = x.cuda(), w.cuda()
+    y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    nb = mq.mq_workspace_bytes(M, K)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    torch.cuda.synchronize()
+    W = mq.Weight(wd)
+    mq.mq_decode_linear_nvfp4(W.handle, xd, M, y, ws, nb)
+    torch.cuda.synchronize()
+    yr, pr = oracle_prefill_rows(x, w, np.arange(M))
+    assert_close(y.cpu(), yr, pr, "nvfp4 decode right after packing")
+    W.free()
+    assert mq.mq_check() == 0
+
+
 def test_decode_paths_share_scratch():
     """BF16 and NVFP4 decode on one split-K handle, alternating: each leaves
     the shared counters at zero for the other, and every round gives the same
