@@ -74,6 +74,18 @@ def test_two_rank_amax_exchange_gloo():
         assert sf == sf_full[r0:r1].tobytes()
 
 
+def test_shard_workspace_sizes():
+    """A shard's buffers: codes [M, K/2], the swizzled scales of M rows (rows
+    padded to 128), the partial maxima and the one float that is exchanged."""
+    from nvfp4_quantized_prefill_b200 import binding as mq
+    from nvfp4_quantized_prefill_b200 import sharded
+    ws = sharded.ShardWorkspace.create(37, 320, device="cpu")
+    assert ws.codes.shape == (37, 160)
+    assert ws.sf.numel() == mq.mq_sf_bytes(37, 320) == 128 * 20
+    assert ws.partials.numel() == mq.MQ_AMAX_PARTIALS_MAX
+    assert ws.amax.numel() == 1 and ws.s_enc.numel() == 1
+
+
 @pytest.mark.gpu
 def test_token_shards_on_one_gpu_bit_identical():
     from mqtest import ensure_built
