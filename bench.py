@@ -28,6 +28,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import torch
@@ -87,12 +88,12 @@ class ClockSampler:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        self.path = None   # a temporary file, made when sampling starts
 
     def __enter__(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.fh = open(self.path, "w")
+            fd, self.path = tempfile.mkstemp(prefix=f"mq_clocks_rank{self.index}_", suffix=".csv")
+            self.fh = os.fdopen(fd, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={CLOCK_QUERY}",
                  "--format=csv,noheader,nounits", "-lms", "200"],
@@ -115,6 +116,11 @@ class ClockSampler:
             rows = [l.split(",") for l in open(self.path) if l.strip()]
         except Exception:
             return None
+        finally:
+            try:
+                os.remove(self.path)
+            except OSError:
+                pass
         if not rows:
             return None
         num = lambda v: v.strip().replace(".", "", 1).isdigit()

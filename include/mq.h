@@ -212,7 +212,11 @@ mq_status mq_prefill_mlp_swiglu_nvfp4(const mq_weight *w_gate_up, const mq_weigh
  * Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
  *
  * The first call on a device looks up the array's device address (with that
- * device current); make that first call before any stream capture begins.
+ * device current) and keeps it for that device's context; the first call
+ * after a cudaDeviceReset looks it up again, since the new context may place
+ * the library's device memory elsewhere.  Make each such first call before
+ * any stream capture begins; a lookup that fails returns MQ_ERR_CUDA and
+ * queues no work.
  * All calls on a device share the one array and it keeps the last call's
  * contents (every byte a call reads is written earlier in the same call, so
  * nothing needs clearing).  Calls whose work overlaps on the GPU -- on two

@@ -44,10 +44,44 @@ struct DeviceInfo {
     bool supported = false;
     int num_sms = 0;
     unsigned *err = nullptr;
+    unsigned long long err_ctx = 0;  // context in which `err` was looked up
 };
 
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+// Process-unique id of the calling thread's current CUDA context, or 0 if
+// there is none.  A device's primary context made anew after cudaDeviceReset
+// has a new id, and with it the library's device image (its __device__
+// arrays) may sit at new addresses, so addresses looked up once per device
+// are cached together with this id.
+unsigned long long current_context_id() {
+    struct Fns {
+        CtxGetCurrentFn get = nullptr;
+        CtxGetIdFn id = nullptr;
+    };
+    static const Fns fns = []() {
+        Fns f;
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            f.get = reinterpret_cast<CtxGetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            f.id = reinterpret_cast<CtxGetIdFn>(p);
+        return f;
+    }();
+    CUcontext c = nullptr;
+    if (!fns.get || !fns.id || fns.get(&c) != CUDA_SUCCESS || !c) return 0;
+    unsigned long long id = 0;
+    if (fns.id(c, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
 
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
@@ -65,14 +99,19 @@ mq_status device_info(DeviceInfo **out) {
             cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return MQ_ERR_CUDA;
         d.supported = (major == 10 && minor == 0);
-        if (d.supported) {
-            void *p = nullptr;
-            if (cudaGetSymbolAddress(&p, g_mq_device_error) != cudaSuccess) return MQ_ERR_CUDA;
-            d.err = static_cast<unsigned *>(p);
-        }
         d.init = true;
     }
     if (!d.supported) return MQ_ERR_UNSUPPORTED_DEVICE;
+    // the error word's device address, once per device context (looked up
+    // again after the context was reset); the lookup itself makes the
+    // context current if it was not
+    const unsigned long long ctx = current_context_id();
+    if (!d.err || ctx == 0 || ctx != d.err_ctx) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_mq_device_error) != cudaSuccess || !p) return MQ_ERR_CUDA;
+        d.err = static_cast<unsigned *>(p);
+        d.err_ctx = current_context_id();
+    }
     *out = &d;
     return MQ_OK;
 }
@@ -532,17 +571,23 @@ static __device__ __align__(256) uint8_t g_mq_noalloc_scratch[MQ_NOALLOC_SCRATCH
 namespace {
 
 uint8_t *g_noalloc_ptr[kMaxDevices];
+unsigned long long g_noalloc_ctx[kMaxDevices];  // context of each cached address
 std::mutex g_noalloc_mu;
 
+// The array's device address on the current device, looked up once per
+// device context (again after a cudaDeviceReset, whose new context may place
+// the library's device image elsewhere).
 mq_status noalloc_scratch(uint8_t **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MQ_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
+    const unsigned long long ctx = current_context_id();
+    if (!g_noalloc_ptr[dev] || ctx == 0 || ctx != g_noalloc_ctx[dev]) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_mq_noalloc_scratch) != cudaSuccess || !p)
             return MQ_ERR_CUDA;
         g_noalloc_ptr[dev] = static_cast<uint8_t *>(p);
+        g_noalloc_ctx[dev] = current_context_id();
     }
     *out = g_noalloc_ptr[dev];
     return MQ_OK;

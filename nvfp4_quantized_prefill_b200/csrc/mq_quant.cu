@@ -83,17 +83,22 @@ __global__ void __launch_bounds__(kThreads, kAmaxBlocksPerSm)
     __shared__ float red[kThreads / 32];
     griddep_wait();
     griddep_launch_dependents();
+    // total < 2^32 - 1 (checked on the host); the loop steps only while the
+    // next start is still below total, so no index ever wraps around 2^32
     const uint32_t total = M * vpr;
     const uint32_t stride = gridDim.x * kThreads;
+    const uint32_t step = kAmaxUnroll * stride;
     const bool dense = ldv == vpr;
     uint32_t mx = 0;
-    for (uint32_t i = blockIdx.x * kThreads + threadIdx.x; i < total; i += kAmaxUnroll * stride) {
+    for (uint32_t i = blockIdx.x * kThreads + threadIdx.x; i < total;
+         i = (total - i > step) ? i + step : total) {
         uint4 v[kAmaxUnroll];
 #pragma unroll
         for (int u = 0; u < kAmaxUnroll; ++u) {
+            // idx is used only when it is below total (no wrap-around)
             const uint32_t idx = i + u * stride;
             v[u] = make_uint4(0, 0, 0, 0);
-            if (idx < total) {
+            if (total - i > static_cast<uint32_t>(u) * stride) {
                 uint64_t off = idx;
                 if (!dense) {
                     const uint32_t r = idx / vpr;

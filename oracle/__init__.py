@@ -198,21 +198,6 @@ def sf_unswizzle(swz: np.ndarray, rows: int, kblocks: int) -> np.ndarray:
     return out
 
 
-def dequantize(codes: np.ndarray, sf: np.ndarray, s_enc: float) -> np.ndarray:
-    """Real-valued NVFP4 matrix e2m1 * dec(sb) / s_enc in float64 (vectorised
-    table lookup; used by tests to build brute-force references)."""
-    lut2 = np.array([e2m1_decode(c) for c in range(16)], dtype=np.float64)
-    lut8 = np.array([e4m3_decode(b) for b in range(256)], dtype=np.float64)
-    rows = codes.shape[0]
-    lo = lut2[codes & 15]
-    hi = lut2[codes >> 4]
-    vals = np.empty((rows, codes.shape[1] * 2), dtype=np.float64)
-    vals[:, 0::2] = lo
-    vals[:, 1::2] = hi
-    scales = np.repeat(lut8[sf], 16, axis=1)
-    return vals * scales / float(s_enc)
-
-
 # -- GEMM, decode, SwiGLU -------------------------------------------------------
 
 def gemm_nvfp4(a_codes, a_sf, a_s_enc, b_codes, b_sf, b_s_enc, rows=None):

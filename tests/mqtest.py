@@ -88,3 +88,18 @@ def fetch_device(ptr: int, nbytes: int) -> np.ndarray:
     torch.cuda.synchronize()
     src = torch.as_tensor(_DevBuf(ptr, nbytes), device="cuda")
     return src.clone().cpu().numpy()
+
+
+def check_h_from_gu(y, h, I, what):
+    """h (BF16) against the oracle's SwiGLU of the GPU's own BF16 gate / up
+    halves of y: within one BF16 ulp, and almost always identical."""
+    g, u = y[:, :I].contiguous(), y[:, I:].contiguous()
+    href = oracle.swiglu(g, u)
+    hg = u16(h)
+    # expf differs between the C library and CUDA by an ulp or so in FP32;
+    # after rounding to BF16 that is at most one BF16 ulp, and rarely.
+    a = bf16_from_u16(hg).double()
+    b = bf16_from_u16(href).double()
+    ulp = torch.clamp(b.abs(), min=2.0 ** -126) * 2.0 ** -7
+    assert ((a - b).abs() <= ulp).all(), what
+    assert (hg == href).mean() > 0.995, what

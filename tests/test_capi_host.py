@@ -101,3 +101,21 @@ def test_new_entry_points_reject_bad_arguments_on_the_host(lib):
     assert L.mq_amax_combine(16, 0, 16, None) == 1
     assert L.mq_amax_combine(16, 4097, 16, None) == 1
     assert L.mq_amax_combine(18, 4, 16, None) == 3
+
+
+def test_amax_shape_bound_at_the_32_bit_edge(lib):
+    """The amax kernel indexes the [M, K/8] vectors with 32-bit unsigned
+    arithmetic, so the host accepts M * K / 8 < 2^32 - 1 and nothing larger.
+    Just below the edge the call gets past the shape check and stops at the
+    (deliberately misaligned) partials pointer; at the edge it is a shape
+    error.  Neither reaches the device."""
+    L = lib
+    n = ctypes.c_int()
+    below = (1 << 29) - 1          # M * 64 / 8 = 2^32 - 8
+    assert below * 8 < (1 << 32) - 1
+    assert L.mq_tensor_amax(16, below, 64, 64, 20, ctypes.byref(n), None) == 3
+    assert L.mq_tensor_amax(16, 1 << 29, 64, 64, 20, ctypes.byref(n), None) == 2
+    # the same edge with longer rows: K = 4096 -> 512 vectors a row
+    rows = ((1 << 32) - 2) // 512  # largest M with M * 512 < 2^32 - 1
+    assert L.mq_tensor_amax(16, rows, 4096, 4096, 20, ctypes.byref(n), None) == 3
+    assert L.mq_tensor_amax(16, rows + 1, 4096, 4096, 20, ctypes.byref(n), None) == 2

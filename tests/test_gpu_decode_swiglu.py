@@ -5,7 +5,8 @@ import pytest
 import torch
 
 import oracle
-from mqtest import (assert_close, bf16_from_u16, ensure_built, gpu_quantize, oracle_prefill_rows,
+from mqtest import (assert_close, bf16_from_u16, check_h_from_gu, ensure_built, gpu_quantize,
+                    oracle_prefill_rows,
                     sample_rows, u16)
 from nvfp4_quantized_prefill_b200 import binding as mq
 from nvfp4_quantized_prefill_b200 import workloads
@@ -93,25 +94,12 @@ def _swiglu_case(M, K, I, seed):
     return x, wgu, Wgu, y.cpu(), h.cpu(), float(part[:n].max())
 
 
-def _check_h_from_gu(y, h, I, what):
-    g, u = y[:, :I].contiguous(), y[:, I:].contiguous()
-    href = oracle.swiglu(g, u)
-    hg = u16(h)
-    # expf differs between the C library and CUDA by an ulp or so in FP32;
-    # after rounding to BF16 that is at most one BF16 ulp, and rarely.
-    a = bf16_from_u16(hg).double()
-    b = bf16_from_u16(href).double()
-    ulp = torch.clamp(b.abs(), min=2.0 ** -126) * 2.0 ** -7
-    assert ((a - b).abs() <= ulp).all(), what
-    assert (hg == href).mean() > 0.995, what
-
-
 @pytest.mark.parametrize("M,K,I", [(200, 256, 256), (128, 512, 384), (1, 64, 128)])
 def test_swiglu_epilogue_small(M, K, I):
     x, wgu, Wgu, y, h, hmax = _swiglu_case(M, K, I, 3)
     yr, pr = oracle_prefill_rows(x, wgu, np.arange(M))
     assert_close(y, yr, pr, "gate/up")
-    _check_h_from_gu(y, h, I, "swiglu")
+    check_h_from_gu(y, h, I, "swiglu")
     assert hmax == float(h.float().abs().max())
     Wgu.free()
     assert mq.mq_check() == 0
@@ -167,7 +155,7 @@ def test_mlp_prefill_llama8b_sampled_rows():
     r = torch.from_numpy(rows)
     gur, gpr = oracle_prefill_rows(x, wgu, rows)
     assert_close(gu[r].cpu(), gur, gpr, "llama8b gate/up")
-    _check_h_from_gu(gu[r].cpu(), h[r].cpu(), I, "llama8b swiglu")
+    check_h_from_gu(gu[r].cpu(), h[r].cpu(), I, "llama8b swiglu")
     # down projection: oracle on the GPU's h (its full-tensor scale)
     hc = h.cpu()
     yr, pr = oracle_prefill_rows(hc, wd, rows)

@@ -6,7 +6,8 @@ import pytest
 import torch
 
 import oracle
-from mqtest import (assert_close, ensure_built, gpu_quantize, oracle_prefill_rows, sample_rows)
+from mqtest import (assert_close, check_h_from_gu, ensure_built, gpu_quantize, oracle_prefill_rows,
+                    sample_rows)
 from nvfp4_quantized_prefill_b200 import binding as mq
 from nvfp4_quantized_prefill_b200 import workloads
 
@@ -131,3 +132,84 @@ def test_prefill_chunk_16384_tokens_sampled():
         ys = y[torch.from_numpy(rows)][:, torch.from_numpy(cols)].cpu()
         assert_close(ys, yr, pr, f"chunk {wl.linears[i].name}")
         W.free()
+
+
+# Llama-3-70B-shaped layer at 16384 tokens: the deepest K (down, K = 28672:
+# 112 K steps of 256 per tile) and the widest N (gate+up, N = 57344) the
+# library runs.  The inputs are drawn with the workload's recipes on the GPU's
+# generator (same distributions, so the 470M-element tensors take seconds) and
+# copied to the host for the oracle; sampled rows x sampled columns keep the
+# oracle's exact sum to seconds.
+_L70 = workloads.WORKLOADS["llama3_70b_layer"]
+
+
+def _gpu_inputs_70b(i: int, K: int):
+    lin = _L70.linears[i]
+    w = workloads.weight(lin.N, lin.K, lin.std, _L70.seed, 100 + i, device="cuda")
+    x = workloads.activation(_L70.act, _L70.M, K, _L70.seed, i, device="cuda")
+    return x, w
+
+
+def _prefill_dev(x: torch.Tensor, W: "mq.Weight") -> torch.Tensor:
+    M, K = x.shape
+    y = torch.empty(M, W.N, dtype=torch.bfloat16, device="cuda")
+    nb = mq.mq_workspace_bytes(M, K)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    mq.mq_prefill_linear_nvfp4(W.handle, x, M, y, ws, nb)
+    torch.cuda.synchronize()
+    del ws
+    return y
+
+
+@pytest.mark.parametrize("i", [0, 1, 2, 3], ids=["qkv", "o", "gate_up", "down"])
+def test_prefill_llama70b_shapes_sampled(i):
+    lin = _L70.linears[i]
+    x, w = _gpu_inputs_70b(i, lin.K)
+    W = mq.Weight(w)
+    y = _prefill_dev(x, W)
+    rows = sample_rows(_L70.M, 5, 20 + i)
+    cols = np.sort(np.random.default_rng(30 + i).choice(lin.N, 768, replace=False))
+    cols = np.unique(np.concatenate([cols, [0, 255, 256, lin.N - 1]]))
+    ys = y[torch.from_numpy(rows)][:, torch.from_numpy(cols)].cpu()
+    del y
+    x_cpu, w_cpu = x.cpu(), w.cpu()
+    del x
+    W.free()
+    del w
+    torch.cuda.empty_cache()
+    yr, pr = oracle_prefill_rows(x_cpu, w_cpu, rows, wrows=cols)
+    assert_close(ys, yr, pr, f"llama70b {lin.name} {_L70.M}x{lin.N}x{lin.K}")
+    assert mq.mq_check() == 0
+
+
+def test_swiglu_llama70b_gate_up_sampled():
+    """The 70B gate+up weight (N = 57344) through the fused SwiGLU epilogue:
+    h on sampled rows within one BF16 ulp of SiLU(g) * u of the GPU's g, u,
+    whose sampled columns are within the GEMM bound of the oracle, and the
+    epilogue's partial maxima equal to max |h|."""
+    lin = _L70.linears[2]
+    M, K, I = _L70.M, lin.K, lin.N // 2
+    x, w = _gpu_inputs_70b(2, K)
+    W = mq.Weight(w)
+    codes, sf, s = gpu_quantize(x)
+    c, f = torch.from_numpy(codes).cuda(), torch.from_numpy(sf).cuda()
+    sd = torch.tensor([s], dtype=torch.float32, device="cuda")
+    gu = torch.empty(M, 2 * I, dtype=torch.bfloat16, device="cuda")
+    mq.mq_gemm_nvfp4(c, f, sd, M, W.handle, gu, 2 * I)
+    h = torch.empty(M, I, dtype=torch.bfloat16, device="cuda")
+    part = torch.empty(mq.MQ_AMAX_PARTIALS_MAX, dtype=torch.float32, device="cuda")
+    n = mq.mq_gemm_nvfp4_swiglu(c, f, sd, M, W.handle, h, part)
+    torch.cuda.synchronize()
+    assert float(part[:n].max()) == float(h.float().abs().max())
+    rows = torch.from_numpy(sample_rows(M, 4, 40))
+    gur, hr = gu[rows].cpu(), h[rows].cpu()
+    check_h_from_gu(gur, hr, I, "llama70b swiglu")
+    cols = np.sort(np.random.default_rng(41).choice(2 * I, 768, replace=False))
+    x_cpu, w_cpu = x.cpu(), w.cpu()
+    del gu, h, x
+    W.free()
+    del w
+    torch.cuda.empty_cache()
+    yr, pr = oracle_prefill_rows(x_cpu, w_cpu, rows.numpy(), wrows=cols)
+    assert_close(gur[:, torch.from_numpy(cols)], yr, pr, "llama70b gate/up")
+    assert mq.mq_check() == 0

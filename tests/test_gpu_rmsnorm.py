@@ -1,6 +1,6 @@
 """GPU parity of the RMSNorm that emits the quantizer's amax, and of the
 prefill linear fed by it: the normalised rows against the oracle's binary64
-RMSNorm (one BF16 step at most, nearly all identical), the NVFP4 codes of the
+RMSNorm (two BF16 steps at most, nearly all identical), the NVFP4 codes of the
 GPU's rows bit-exact, the GEMM within tolerance."""
 import numpy as np
 import pytest

@@ -5,8 +5,9 @@ scales and outputs are the single-GPU ones bit for bit.
 CPU (gloo, 2 ranks): the exchange of nvfp4_quantized_prefill_b200.sharded
 (all-reduce max of one float) with the oracle doing each rank's amax and
 quantization.  GPU: the library's shard halves run for several shards in one
-process (the exchange being the max of the shards' floats), against the
-single-call prefill linear."""
+process (the exchange being the max of the shards' floats); each shard's
+outputs are compared with the oracle's prefill of the whole batch, and all of
+them together with the single-call prefill linear."""
 import os
 import socket
 import sys
@@ -114,6 +115,14 @@ def test_token_shards_on_one_gpu_bit_identical():
         sharded.shard_finish(W, t, y, w)
     torch.cuda.synchronize()
     assert float(amax) == oracle.tensor_amax(x)
+    # every shard's rows against the oracle's prefill of the whole batch (the
+    # batch's tensor scales), at the GEMM tolerance
+    from mqtest import assert_close, oracle_prefill_rows
+    w_cpu = workloads.weight(N, K, 0.02, 9, 1)
+    for (a, b), y in zip(zip(bounds, bounds[1:]), ys):
+        y_or, p_or = oracle_prefill_rows(x, w_cpu, np.arange(a, b))
+        assert_close(y.cpu(), y_or, p_or, f"token shard rows {a}..{b}")
+    # and the shards together reproduce the single-call prefill bit for bit
     assert torch.equal(torch.cat(ys).view(torch.int16), y_full.view(torch.int16))
     W.free()
     assert mq.mq_check() == 0

@@ -3,8 +3,9 @@
 It exists for callers that cannot allocate device memory (a plugin handed
 only its input and output buffers, or a latency-critical path that must not
 pay the device synchronization of cudaMalloc / cudaFree): its scratch is a
-fixed array inside the library's device image.  This file is collected last
-so that a run stopping at the first failure has already run everything else.
+fixed array inside the library's device image, shared by every call.  This
+file is collected last so that a run stopping at the first failure has
+already run everything else.
 """
 import numpy as np
 import pytest
@@ -25,27 +26,42 @@ def _existing(W, x, M):
     return y
 
 
-def test_noalloc_matches_workspace_entry_on_two_calls_in_a_row():
-    ensure_built()
-    # two different problems back to back through the shared scratch: the
-    # second must not see anything the first left behind
-    cases = [(300, 520, 512, 0), (1000, 768, 256, 1)]
-    for M, N, K, seed in cases:
-        x_cpu = workloads.activation("outlier", M, K, seed, 0)
+def _check_sequence(cases):
+    """Runs the cases back to back through the one shared scratch array.
+    Each output must equal the workspace entry point's bit for bit (same
+    kernels, same inputs) and be within the GEMM tolerance of the oracle."""
+    for M, N, K, seed, recipe in cases:
+        x_cpu = workloads.activation(recipe, M, K, seed, 0)
         w_cpu = workloads.weight(N, K, 0.02, seed, 1)
         W = mq.Weight(w_cpu.cuda())
         x = x_cpu.cuda()
-        y_ref = _existing(W, x, M)
         y_new = torch.full((M, N), 3.0, dtype=torch.bfloat16, device="cuda")
         mq.mq_prefill_linear_nvfp4_noalloc(W.handle, x, M, y_new)
+        y_ref = _existing(W, x, M)
         torch.cuda.synchronize()
         assert mq.mq_check() == 0
-        # the same tolerance as every GEMM parity test, with the oracle's
-        # sum of |products| for the bound
-        _, p_ref = oracle_prefill_rows(x_cpu, w_cpu, np.arange(M))
-        ref = y_ref.float().cpu().double().numpy()
-        assert_close(y_new.cpu(), ref, p_ref, f"noalloc vs workspace entry {M}x{N}x{K}")
+        assert torch.equal(y_new.view(torch.int16), y_ref.view(torch.int16)), (
+            f"noalloc differs from the workspace entry point at {M}x{N}x{K}")
+        y_or, p_or = oracle_prefill_rows(x_cpu, w_cpu, np.arange(M))
+        assert_close(y_new.cpu(), y_or, p_or, f"noalloc vs oracle {M}x{N}x{K}")
         W.free()
+
+
+def test_noalloc_matches_workspace_entry_and_oracle_on_two_calls_in_a_row():
+    ensure_built()
+    # two different problems back to back: the second must not see anything
+    # the first left behind
+    _check_sequence([(300, 520, 512, 0, "outlier"), (1000, 768, 256, 1, "outlier")])
+
+
+def test_noalloc_small_ragged_call_after_a_large_one():
+    ensure_built()
+    # the large call fills far more of the array (codes, scale tiles with
+    # their padding rows, partial maxima, tensor scale) than the ragged call
+    # after it writes, with a different scale, so stale bytes from the first
+    # sit right after and inside the second call's region
+    _check_sequence([(1500, 384, 1024, 3, "student_t3"), (77, 200, 320, 4, "outlier"),
+                     (129, 256, 64, 5, "channel_gain")])
 
 
 def test_noalloc_rejects_requests_larger_than_its_scratch():
