@@ -318,27 +318,61 @@ class Prefill:
                                  lambda st, q=q, W=W, y=y: mq.mq_gemm_nvfp4(
                                      q["codes"], q["sf"], q["s"], M, W.handle, y, W.N, st)))
                 self.flops += 2.0 * M * W.N * W.K
-        # decode (phase switch) on every weight handle at M = 1
-        self.dec = []
-        xdec = self.xs[0][:1].contiguous()
-        for W in self.W:
-            xd = xdec if W.K == xdec.shape[1] else torch.zeros(1, W.K, dtype=bf, device=dev)
-            yd = torch.empty(1, W.N, dtype=bf, device=dev)
-            self.dec.append(lambda st, W=W, xd=xd, yd=yd: mq.mq_decode_linear_bf16(
-                W.handle, xd, 1, yd, st))
-        self.decode_bytes = sum(2.0 * W.N * W.K + 2.0 * W.K + 2.0 * W.N for W in self.W)
-        # uniform-NVFP4 (W4A4) decode on the same handles: x quantized per call
-        self.dec4 = []
-        for W in self.W:
-            xd = xdec if W.K == xdec.shape[1] else torch.zeros(1, W.K, dtype=bf, device=dev)
-            yd = torch.empty(1, W.N, dtype=bf, device=dev)
-            nb = mq.mq_workspace_bytes(1, W.K)
-            ws4 = torch.empty(nb, dtype=torch.uint8, device=dev)
-            self.dec4.append(lambda st, W=W, xd=xd, yd=yd, ws4=ws4, nb=nb: mq.mq_decode_linear_nvfp4(
-                W.handle, xd, 1, yd, ws4, nb, st))
-        # weight codes + E4M3 scales (0.5625 byte per parameter) and x / y
-        self.decode4_bytes = sum(0.5625 * W.N * W.K + 2.0 * W.K + 2.0 * W.N for W in self.W)
+        # decode (phase switch) on every weight handle at M = 1: BF16, and
+        # uniform NVFP4 (W4A4, tokens quantized inside the call) for comparison
+        self.dec, self.decode_bytes = self.decode_calls(1, "bf16")
+        self.dec4, self.decode4_bytes = self.decode_calls(1, "nvfp4")
         self.launches = len(self.ops) + len(self.dec)   # one kernel per op / decode call
+
+    def decode_calls(self, Md: int, kind: str):
+        """Decode of Md tokens on every weight handle (the first activation's
+        first rows where K matches, zeros otherwise).  Returns (launch
+        closures, bytes moved per pass: the weight at 2 (BF16) or 0.5625
+        (NVFP4 codes + E4M3 scales) bytes per parameter, plus x and y)."""
+        mq, dev, bf = self.mq, self.dev, torch.bfloat16
+        calls, nbytes = [], 0.0
+        x0 = self.xs[0][:Md].contiguous()
+        for W in self.W:
+            xd = x0 if W.K == x0.shape[1] else torch.zeros(Md, W.K, dtype=bf, device=dev)
+            yd = torch.empty(Md, W.N, dtype=bf, device=dev)
+            if kind == "bf16":
+                calls.append(lambda st, W=W, xd=xd, yd=yd: mq.mq_decode_linear_bf16(
+                    W.handle, xd, Md, yd, st))
+                nbytes += 2.0 * W.N * W.K
+            else:
+                nb = mq.mq_workspace_bytes(Md, W.K)
+                ws4 = torch.empty(nb, dtype=torch.uint8, device=dev)
+                calls.append(lambda st, W=W, xd=xd, yd=yd, ws4=ws4, nb=nb:
+                             mq.mq_decode_linear_nvfp4(W.handle, xd, Md, yd, ws4, nb, st))
+                nbytes += 0.5625 * W.N * W.K
+            nbytes += 2.0 * Md * W.K + 2.0 * Md * W.N
+        return calls, nbytes
+
+    def run_bf16(self):
+        """The same-shape BF16 path (cuBLAS through torch.matmul; SiLU * up in
+        torch for MLPs): the comparator of the speedup, not part of the library."""
+        wl, P = self.wl, self
+        if wl.swiglu:
+            for item in P.plan:
+                if item[0] == "mlp":
+                    _, i, j, xi = item
+                    gu = torch.matmul(P.xs[xi], P.ws[i].t())
+                    I = gu.shape[1] // 2
+                    h = torch.nn.functional.silu(gu[:, :I]) * gu[:, I:]
+                    torch.matmul(h, P.ws[j].t())
+                else:
+                    _, i, xi = item
+                    torch.matmul(P.xs[xi], P.ws[i].t())
+        elif wl.chunks > 1:
+            for x in P.xs:
+                for w in P.ws:
+                    torch.matmul(x, w.t())
+        else:
+            for i, (x, w) in enumerate(zip(P.xs, P.ws)):
+                if wl.rmsnorm and i == 0:
+                    r, gain = P.rs[0]
+                    x = torch.nn.functional.rms_norm(r, (r.shape[1],), weight=gain, eps=RMS_EPS)
+                torch.matmul(x, w.t())
 
     def _add_quant(self, name, x, K, q):
         mq, M = self.mq, self.M
@@ -363,6 +397,100 @@ class Prefill:
     def free(self):
         for W in self.W:
             W.free()
+
+
+# workloads measured next to the headline one (each in its own Prefill, freed
+# before the next): the 8B SwiGLU MLP with decode at 1 and 8 tokens, the
+# chunked 131072-token prefill and the 70B layer's linears
+PER_CONFIG = ("llama3_8b_mlp", "chunked_131k", "llama3_70b_layer")
+
+
+def measure_light(key, args, mq, dev, stream, flush, capture, replay_ms, pk):
+    """One workload's prefill timed like the headline (CUDA events at the step
+    boundaries, L2 flushed between steps, kernels chained by programmatic
+    dependent launch), the GEMM-only rate from a pass with an event after
+    every launch, the cuBLAS BF16 comparator, and decode device times from
+    CUDA-graph replays.  Returns a dict for the bench line's per_config."""
+    wl = workloads.WORKLOADS[key]
+    P = Prefill(wl, mq, dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    steps, warm = args.config_steps, max(3, args.warmup)
+    for _ in range(warm):
+        flush()
+        P.run_prefill(stream)
+    torch.cuda.synchronize()
+    if mq.mq_check(stream) != 0:
+        raise RuntimeError(f"device error in {key}")
+    pairs = [(ev(), ev()) for _ in range(steps)]
+    for a, b in pairs:
+        flush()
+        a.record(stream)
+        P.run_prefill(stream)
+        b.record(stream)
+    torch.cuda.synchronize()
+    t_ms = sum(a.elapsed_time(b) for a, b in pairs) / steps
+    # GEMM launches alone (events between launches)
+    gemm_ms = 0.0
+    for _ in range(2):
+        flush()
+        evs = [ev() for _ in range(len(P.ops) + 1)]
+        evs[0].record(stream)
+        for i, (_, _, f) in enumerate(P.ops):
+            f(stream)
+            evs[i + 1].record(stream)
+        torch.cuda.synchronize()
+        gemm_ms += sum(evs[i].elapsed_time(evs[i + 1]) for i, o in enumerate(P.ops)
+                       if o[1] == "gemm") / 2
+    bts = []
+    P.run_bf16()
+    for _ in range(3):
+        flush()
+        a, b = ev(), ev()
+        a.record(stream)
+        P.run_bf16()
+        b.record(stream)
+        torch.cuda.synchronize()
+        bts.append(a.elapsed_time(b))
+    bf16_ms = statistics.median(bts)
+    fp4_peak = pk["bf16"] * FP4_OVER_BF16
+    tokens = wl.M * max(1, wl.chunks)
+    tf = P.flops / (t_ms * 1e-3) / 1e12
+    r = {"workload": wl.name, "tokens": tokens,
+         "linears": [{"name": l.name, "N": l.N, "K": l.K} for l in wl.linears],
+         "activations": wl.act, "seed": wl.seed, "steps": steps, "warmup": warm,
+         "prefill_ms": round(t_ms, 4), "tflops": round(tf, 2),
+         "fp4_peak_frac": round(tf / fp4_peak, 4),
+         "gemm_only_tflops": round(P.flops / (gemm_ms * 1e-3) / 1e12, 2),
+         "bf16_cublas_ms": round(bf16_ms, 4), "speedup_vs_bf16": round(bf16_ms / t_ms, 3),
+         "tokens_per_s": round(tokens / (t_ms * 1e-3), 1)}
+    if wl.chunks > 1:
+        r["chunks"] = wl.chunks
+        r["per_chunk_ms"] = round(t_ms / wl.chunks, 4)
+        r["total_ms"] = round(t_ms, 4)
+    # decode at the workload's token counts: device time per pass from graph
+    # replays of R x (flush, decode of every handle) minus R flushes
+    if len(wl.decode_M) > 1:
+        R = 16
+        t_flush = replay_ms(capture([]))
+        dec = {}
+        for Md in wl.decode_M:
+            for kind in ("bf16", "nvfp4"):
+                calls, nbytes = P.decode_calls(Md, kind)
+                for f in calls:      # first calls outside the capture
+                    f(stream)
+                torch.cuda.synchronize()
+                g = capture(calls)
+                d_ms = (replay_ms(g) - t_flush) / R
+                del g
+                dec[f"{kind}_m{Md}_ms"] = round(d_ms, 4)
+                dec[f"{kind}_m{Md}_gbs"] = round(nbytes / (d_ms * 1e-3) / 1e9, 1)
+        r["decode"] = dec
+        r["decode_note"] = ("device time per pass over every handle (graph replays, L2 flushed "
+                            "before each pass); GB/s over the weight bytes (2 or 0.5625 B/param) "
+                            "+ x + y; nvfp4 = W4A4 with the tokens quantized inside the call")
+    P.free()
+    del P
+    return r
 
 
 def run_gpu(args, wl, world, rank):
@@ -542,28 +670,7 @@ def run_gpu(args, wl, world, rank):
     # ---- the same-shape BF16 path (cuBLAS through torch.matmul): comparator only
     bf16_ms = None
     try:
-        def bf16_prefill():
-            if wl.swiglu:
-                for item in P.plan:
-                    if item[0] == "mlp":
-                        _, i, j, xi = item
-                        gu = torch.matmul(P.xs[xi], P.ws[i].t())
-                        I = gu.shape[1] // 2
-                        h = torch.nn.functional.silu(gu[:, :I]) * gu[:, I:]
-                        torch.matmul(h, P.ws[j].t())
-                    else:
-                        _, i, xi = item
-                        torch.matmul(P.xs[xi], P.ws[i].t())
-            elif wl.chunks > 1:
-                for x in P.xs:
-                    for w in P.ws:
-                        torch.matmul(x, w.t())
-            else:
-                for i, (x, w) in enumerate(zip(P.xs, P.ws)):
-                    if wl.rmsnorm and i == 0:
-                        r, gain = P.rs[0]
-                        x = torch.nn.functional.rms_norm(r, (r.shape[1],), weight=gain, eps=RMS_EPS)
-                    torch.matmul(x, w.t())
+        bf16_prefill = P.run_bf16
         bf16_prefill()
         bt = []
         for _ in range(max(3, min(args.steps, 10))):
@@ -670,6 +777,21 @@ def run_gpu(args, wl, world, rank):
                "path": "mq_prefill_linear_nvfp4 per projection; pinned-host X in and Y out "
                        "on their own streams, overlapping each other and the compute"}
 
+    # ---- the other workloads, lighter: prefill TFLOP/s incl. quantization,
+    # GEMM-only TFLOP/s, the BF16 comparator, tokens/s, and decode at the
+    # workload's token counts (BF16 and W4A4)
+    per_config = None
+    if args.per_config and world == 1:
+        per_config = {}
+        for key in PER_CONFIG:
+            if key == args.workload:
+                continue
+            per_config[key] = measure_light(key, args, mq, dev, stream, flush, capture,
+                                            replay_ms, pk)
+            torch.cuda.empty_cache()
+        if mq.mq_check(stream) != 0:
+            raise RuntimeError("device error during the per-workload measurements")
+
     traffic, traffic_launches = recorded_traffic(args.workload)
     clk = clocks.summary()
     out = {
@@ -746,6 +868,7 @@ def run_gpu(args, wl, world, rank):
         "e2e": e2e,
         "gpu_launches": P.launches * args.steps,
         "clocks": clk,
+        **({"per_config": per_config} if per_config is not None else {}),
     }
     return out, P
 
@@ -760,6 +883,10 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=32,
                     help="activation rows per projection in the CPU oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", dest="per_config", action="store_false",
+                    help="skip the lighter measurement of the other workloads")
+    ap.add_argument("--config-steps", type=int, default=5,
+                    help="timed steps per workload in per_config")
     args = ap.parse_args()
     wl = workloads.WORKLOADS[args.workload]
 
