@@ -79,6 +79,9 @@ def _load():
             lib.mqo_double_to_bf16_rne.argtypes = [ctypes.c_double]
             lib.mqo_rmsnorm.restype = None
             lib.mqo_rmsnorm.argtypes = [P, I64, I64, I64, P, ctypes.c_double, P]
+            lib.mqo_attention.restype = None
+            lib.mqo_attention.argtypes = [P, I64, P, I64, I64, P, I64, I64, I64, I64, I64, I64,
+                                          ctypes.c_double, P, I64, P, P]
             lib.mqo_set_threads.restype = None
             lib.mqo_set_threads.argtypes = [ctypes.c_int]
             lib.mqo_threads_used.restype = ctypes.c_int
@@ -255,3 +258,25 @@ def rmsnorm(x, gamma, eps: float) -> np.ndarray:
     y = np.zeros((rows, cols), dtype=np.uint16)
     _load().mqo_rmsnorm(_ptr(xa), rows, cols, cols, _ptr(ga), float(eps), _ptr(y))
     return y
+
+
+# -- attention of the prefill layer / decode step ------------------------------
+
+def attention(q, k, v, H: int, Hkv: int, D: int, pos0: int = 0, rows=None, scale=None):
+    """Causal grouped-query softmax attention in binary64 (mqo_attention).
+
+    q: BF16 [n_q, H*D] (query i at absolute position pos0 + i); k, v: BF16
+    [n_k, Hkv*D] with n_k >= pos0 + n_q (key j at position j).  Returns
+    (o float64 [len(rows), H, D], a float64 [len(rows), H, D]) for the query
+    rows (all if None); a = the softmax-weighted |v|."""
+    qa, ka, va = _u16(q), _u16(k), _u16(v)
+    n_q = qa.shape[0]
+    assert qa.shape[1] == H * D and ka.shape[1] == Hkv * D and va.shape[1] == Hkv * D
+    assert ka.shape[0] >= pos0 + n_q and va.shape[0] >= pos0 + n_q and H % Hkv == 0
+    idx = np.arange(n_q, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    out = np.zeros((idx.size, H, D), dtype=np.float64)
+    a = np.zeros((idx.size, H, D), dtype=np.float64)
+    sc = (1.0 / np.sqrt(D)) if scale is None else float(scale)
+    _load().mqo_attention(_ptr(qa), H * D, _ptr(ka), Hkv * D, D, _ptr(va), Hkv * D, D, pos0, H, Hkv,
+                          D, sc, _ptr(idx), idx.size, _ptr(out), _ptr(a))
+    return out, a

@@ -406,3 +406,63 @@ void mqo_rmsnorm(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, cons
         }
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* Attention of the prefill layer and of the decode step                   */
+/* ------------------------------------------------------------------------ */
+
+/* [reading] The pages name the KV cache that prefill builds and decode
+ * consumes (zingnex.cn forum thread, section "动态精度切换"; gist.science
+ * technical summary, section 2 "System-Level Deployment") but do not define
+ * the attention itself.  The plain causal softmax attention of the Llama
+ * family's layer is used, with grouped KV heads and no positional rotation:
+ *
+ *   o[i, h, :] = sum_{j <= pos0 + i} w_j v[j, g, :] / sum_j w_j,
+ *   w_j = exp(s_j - max_j s_j),  s_j = scale * sum_d q[i, h, d] k[j, g, d],
+ *   g = h / (H / Hkv)   (query heads h share KV head g in groups of H/Hkv),
+ *
+ * evaluated in binary64 from the BF16 inputs (each product q k is exact in
+ * binary64).  Query i sits at absolute position pos0 + i; keys 0..pos0+i
+ * are visible to it.  q[i, h, d] is at q[i * q_tok + h * D + d], k[j, g, d]
+ * at k[j * k_tok + g * k_head + d], v likewise.  For the requested query
+ * rows, out[r][h][d] = o and a[r][h][d] = sum_j w_j |v[j, g, d]| / sum_j w_j
+ * (the weighted magnitude that bounds rounding errors of a GPU evaluation). */
+void mqo_attention(const uint16_t *q, int64_t q_tok, const uint16_t *k, int64_t k_tok,
+                   int64_t k_head, const uint16_t *v, int64_t v_tok, int64_t v_head,
+                   int64_t pos0, int64_t H, int64_t Hkv, int64_t D, double scale,
+                   const int64_t *rows, int64_t n_rows, double *out, double *a) {
+    const int64_t group = H / Hkv;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic) num_threads(MQO_NT)
+#endif
+    for (int64_t t = 0; t < n_rows * H; ++t) {
+        const int64_t r = t / H, h = t % H, i = rows[r], g = h / group;
+        const int64_t n_keys = pos0 + i + 1;
+        double *s = (double *)malloc(sizeof(double) * (size_t)n_keys);
+        double smax = -INFINITY;
+        for (int64_t j = 0; j < n_keys; ++j) {
+            double acc = 0.0;
+            for (int64_t d = 0; d < D; ++d)
+                acc += (double)mqo_bf16_to_float(q[i * q_tok + h * D + d]) *
+                       (double)mqo_bf16_to_float(k[j * k_tok + g * k_head + d]);
+            s[j] = scale * acc;
+            if (s[j] > smax) smax = s[j];
+        }
+        double z = 0.0;
+        for (int64_t j = 0; j < n_keys; ++j) {
+            s[j] = exp(s[j] - smax);
+            z += s[j];
+        }
+        for (int64_t d = 0; d < D; ++d) {
+            double o = 0.0, m = 0.0;
+            for (int64_t j = 0; j < n_keys; ++j) {
+                const double vv = (double)mqo_bf16_to_float(v[j * v_tok + g * v_head + d]);
+                o += s[j] * vv;
+                m += s[j] * fabs(vv);
+            }
+            out[(r * H + h) * D + d] = o / z;
+            a[(r * H + h) * D + d] = m / z;
+        }
+        free(s);
+    }
+}

@@ -410,3 +410,92 @@ def test_rmsnorm_matches_torch_library(oracle_mod):
     y = oracle_mod.rmsnorm(x, one, 1e-5)
     ref = torch.nn.functional.rms_norm(x.double(), (512,), eps=1e-5).to(torch.bfloat16)
     assert (y == bf16_bits(ref)).all()
+
+
+# ---------------------------------------------------------------------------
+# attention (prefill layer and decode step)
+# ---------------------------------------------------------------------------
+
+def _qkv(n, H, Hkv, D, seed):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(n, H * D, generator=g).to(torch.bfloat16)
+    k = torch.randn(n, Hkv * D, generator=g).to(torch.bfloat16)
+    v = torch.randn(n, Hkv * D, generator=g).to(torch.bfloat16)
+    return q, k, v
+
+
+def test_attention_first_query_sees_only_the_first_key(oracle_mod):
+    q, k, v = _qkv(6, 4, 2, 16, 1)
+    o, a = oracle_mod.attention(q, k, v, 4, 2, 16)
+    vv = v.double().numpy().reshape(6, 2, 16)
+    for h in range(4):
+        assert np.array_equal(o[0, h], vv[0, h // 2])       # one visible key: exactly v_0
+        assert np.array_equal(a[0, h], np.abs(vv[0, h // 2]))
+
+
+def test_attention_zero_queries_give_running_means(oracle_mod):
+    """q = 0: every visible key weighs the same, o_i = mean(v_0 .. v_i)."""
+    n, H, Hkv, D = 9, 4, 2, 8
+    _, k, v = _qkv(n, H, Hkv, D, 2)
+    q = torch.zeros(n, H * D, dtype=torch.bfloat16)
+    o, _ = oracle_mod.attention(q, k, v, H, Hkv, D)
+    vv = v.double().numpy().reshape(n, Hkv, D)
+    mean = np.cumsum(vv, axis=0) / np.arange(1, n + 1)[:, None, None]
+    for h in range(H):
+        assert np.allclose(o[:, h], mean[:, h // 2], rtol=0, atol=1e-14)
+
+
+def test_attention_dominant_key_selects_its_value(oracle_mod):
+    """k_j = c e_j and q_i = c e_t: key t out-scores every other by c^2/sqrt(D)
+    (= 64 here), so o_i = v_t up to e^-64."""
+    n, D, c = 8, 16, 16.0
+    k = torch.zeros(n, D)
+    for j in range(n):
+        k[j, j] = c
+    q = torch.zeros(n, D)
+    t = 3
+    q[:, t] = c
+    v = torch.randn(n, D, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+    o, _ = oracle_mod.attention(q.to(torch.bfloat16), k.to(torch.bfloat16), v, 1, 1, D)
+    vv = v.double().numpy()
+    for i in range(t, n):
+        assert np.allclose(o[i, 0], vv[t], rtol=0, atol=1e-20 + 1e-25)
+    # before key t is visible the queries score 0 against every key: uniform
+    for i in range(t):
+        assert np.allclose(o[i, 0], vv[: i + 1].mean(axis=0), rtol=0, atol=1e-14)
+
+
+def test_attention_query_heads_read_their_groups_kv_head(oracle_mod):
+    """H = 4 query heads over Hkv = 2 KV heads: heads 0-1 read KV head 0 and
+    heads 2-3 KV head 1 (a mapping like h % Hkv would mix them)."""
+    n, H, Hkv, D = 5, 4, 2, 8
+    q, k, _ = _qkv(n, H, Hkv, D, 4)
+    v = torch.cat([torch.full((n, D), 1.0), torch.full((n, D), 2.0)], dim=1).to(torch.bfloat16)
+    o, a = oracle_mod.attention(q, k, v, H, Hkv, D)
+    assert np.all(o[:, 0:2] == 1.0) and np.all(o[:, 2:4] == 2.0)
+    assert np.array_equal(a, o)                 # v >= 0: the weighted |v| is o itself
+
+
+def test_attention_matches_torch_sdpa_in_binary64(oracle_mod):
+    n, H, Hkv, D = 37, 8, 2, 32
+    q, k, v = _qkv(n, H, Hkv, D, 5)
+    o, a = oracle_mod.attention(q, k, v, H, Hkv, D)
+    qt = q.double().view(n, H, D).transpose(0, 1)
+    kt = k.double().view(n, Hkv, D).transpose(0, 1).repeat_interleave(H // Hkv, dim=0)
+    vt = v.double().view(n, Hkv, D).transpose(0, 1).repeat_interleave(H // Hkv, dim=0)
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=True)
+    ref = ref.transpose(0, 1).numpy()
+    assert np.allclose(o, ref, rtol=1e-12, atol=1e-14)
+    assert np.all(a >= np.abs(o) - 1e-15)
+
+
+def test_attention_decode_rows_equal_prefill_rows(oracle_mod):
+    """New queries at positions S.. over a cache holding keys 0..S+t are the
+    prefill's rows S.. of the concatenated sequence (the phase hand-off)."""
+    n, S, H, Hkv, D = 20, 15, 4, 1, 16
+    q, k, v = _qkv(n, H, Hkv, D, 6)
+    full, _ = oracle_mod.attention(q, k, v, H, Hkv, D)
+    dec, _ = oracle_mod.attention(q[S:], k, v, H, Hkv, D, pos0=S)
+    assert np.array_equal(dec, full[S:])
+    some, _ = oracle_mod.attention(q, k, v, H, Hkv, D, rows=[0, 7, 19])
+    assert np.array_equal(some, full[[0, 7, 19]])
