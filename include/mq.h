@@ -287,6 +287,54 @@ mq_status mq_decode_linear_bf16(const mq_weight *w, const void *x_bf16, int64_t 
 mq_status mq_decode_linear_nvfp4(const mq_weight *w, const void *x_bf16, int64_t M, void *y_bf16,
                                  void *workspace, size_t ws_bytes, cudaStream_t stream);
 
+/* ---- attention of the prefill layer and the KV cache the decode step reads --
+ * Mix-Quant's prefill builds the KV cache that decoding consumes
+ * (gist.science technical summary, section 2 "System-Level Deployment"; the
+ * zingnex.cn forum thread, section "动态精度切换", on the cache kept across
+ * the two precisions).  The pages do not define the attention; the Llama
+ * family's causal softmax attention with grouped KV heads is used, without
+ * positional rotation:
+ *   o[i, h, :] = sum_{j <= pos(i)} softmax_j( q[i,h,:] . k[j,g,:] / sqrt(D) ) v[j,g,:],
+ *   g = h / (H / Hkv).
+ * Head dimension D = 128.  The activations use the QKV projection's output
+ * layout: qkv (device) BF16 [rows, (H + 2 Hkv) * 128], query heads first, then
+ * the Hkv key heads, then the Hkv value heads.  The KV cache is two device
+ * BF16 arrays [Hkv, S_max, 128] (key / value of head g at position j at
+ * (g * S_max + j) * 128), owned by the caller. */
+
+/* Prefill attention over M tokens (positions 0 .. M-1) on the tensor cores
+ * (BF16 products, FP32 softmax and accumulation): writes o (device, BF16
+ * [M, H * 128], the O projection's input), keys and values of positions
+ * 0 .. M-1 into the cache (k_cache / v_cache may both be NULL to skip it;
+ * otherwise M <= S_max), and *n_partials partial maxima of |o| to
+ * o_amax_partials (device, MQ_AMAX_PARTIALS_MAX floats), so the O
+ * projection's quantizer (mq_quantize_nvfp4 with these partials) skips its
+ * amax pass.  *n_partials is set on the host at once.  Requirements: D == 128,
+ * H % Hkv == 0, all pointers 16-byte aligned.  Bounded waits: a timeout is
+ * latched and reported by mq_check. */
+mq_status mq_attention_prefill_bf16(const void *qkv_bf16, int64_t M, int64_t H, int64_t Hkv,
+                                    int64_t D, void *k_cache, void *v_cache, int64_t S_max,
+                                    void *o_bf16, float *o_amax_partials, int *n_partials,
+                                    cudaStream_t stream);
+
+/* Scratch bytes mq_attention_decode_bf16 needs for m new tokens after pos0
+ * cached ones (0 for invalid sizes). */
+size_t mq_attention_decode_workspace_bytes(int64_t m, int64_t pos0, int64_t H, int64_t Hkv,
+                                           int64_t D);
+
+/* Decode-step attention (BF16 cache, FP32 arithmetic) for m new tokens at
+ * positions pos0 .. pos0 + m - 1: appends their keys and values (from qkv,
+ * device BF16 [m, (H + 2 Hkv) * 128], the BF16 decode QKV projection's
+ * output) to the cache, then token t attends over positions 0 .. pos0 + t.
+ * Writes o (device, BF16 [m, H * 128]).  Requirements: D == 128,
+ * H % Hkv == 0, (H / Hkv) * m <= 64, pos0 + m <= S_max, pointers 16-byte
+ * aligned, workspace (device, 16-byte aligned) of at least
+ * mq_attention_decode_workspace_bytes(m, pos0, H, Hkv, D) bytes. */
+mq_status mq_attention_decode_bf16(const void *qkv_bf16, int64_t m, int64_t pos0, int64_t H,
+                                   int64_t Hkv, int64_t D, void *k_cache, void *v_cache,
+                                   int64_t S_max, void *o_bf16, void *workspace, size_t ws_bytes,
+                                   cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -43,6 +43,11 @@ SIGNATURES = [
     ("mq_decode_linear_nvfp4", _I, [_P, _P, _I64, _P, _P, _SZ, _P]),
     ("mq_rmsnorm_amax", _I, [_P, _P, ctypes.c_float, _I64, _I64, _I64, _P, _P, ctypes.POINTER(_I), _P]),
     ("mq_prefill_linear_rmsnorm_nvfp4", _I, [_P, _P, _P, ctypes.c_float, _I64, _P, _P, _P, _SZ, _P]),
+    ("mq_attention_prefill_bf16", _I, [_P, _I64, _I64, _I64, _I64, _P, _P, _I64, _P, _P,
+                                       ctypes.POINTER(_I), _P]),
+    ("mq_attention_decode_workspace_bytes", _SZ, [_I64, _I64, _I64, _I64, _I64]),
+    ("mq_attention_decode_bf16", _I, [_P, _I64, _I64, _I64, _I64, _I64, _P, _P, _I64, _P, _P, _SZ,
+                                      _P]),
 ]
 
 _lib = None
@@ -235,3 +240,24 @@ class Weight:
             self.free()
         except Exception:
             pass
+
+
+def mq_attention_prefill_bf16(qkv, M: int, H: int, Hkv: int, D: int, k_cache, v_cache, S_max: int,
+                              o, o_amax_partials, stream=None) -> int:
+    """Returns the number of partial maxima written."""
+    n = ctypes.c_int()
+    _ok("mq_attention_prefill_bf16", lib().mq_attention_prefill_bf16(
+        _ptr(qkv), M, H, Hkv, D, _ptr(k_cache), _ptr(v_cache), S_max, _ptr(o), _ptr(o_amax_partials),
+        ctypes.byref(n), _stream(stream)))
+    return n.value
+
+
+def mq_attention_decode_workspace_bytes(m: int, pos0: int, H: int, Hkv: int, D: int) -> int:
+    return lib().mq_attention_decode_workspace_bytes(m, pos0, H, Hkv, D)
+
+
+def mq_attention_decode_bf16(qkv, m: int, pos0: int, H: int, Hkv: int, D: int, k_cache, v_cache,
+                             S_max: int, o, workspace, ws_bytes: int, stream=None) -> None:
+    _ok("mq_attention_decode_bf16", lib().mq_attention_decode_bf16(
+        _ptr(qkv), m, pos0, H, Hkv, D, _ptr(k_cache), _ptr(v_cache), S_max, _ptr(o), _ptr(workspace),
+        ws_bytes, _stream(stream)))

@@ -654,6 +654,59 @@ mq_status mq_decode_linear_nvfp4(const mq_weight *w, const void *x_bf16, int64_t
                                               d->num_sms, stream));
 }
 
+mq_status mq_attention_prefill_bf16(const void *qkv_bf16, int64_t M, int64_t H, int64_t Hkv,
+                                    int64_t D, void *k_cache, void *v_cache, int64_t S_max,
+                                    void *o_bf16, float *o_amax_partials, int *n_partials,
+                                    cudaStream_t stream) {
+    if (!qkv_bf16 || !o_bf16 || !o_amax_partials || !n_partials) return MQ_ERR_INVALID_ARG;
+    if ((k_cache == nullptr) != (v_cache == nullptr)) return MQ_ERR_INVALID_ARG;
+    if (D != 128 || H < 1 || Hkv < 1 || H % Hkv != 0 || M < 1 || M > (1LL << 24) || H > 1024)
+        return MQ_ERR_SHAPE;
+    if (k_cache && (S_max < M || S_max > (1LL << 24))) return MQ_ERR_SHAPE;
+    if (!aligned16(qkv_bf16) || !aligned16(o_bf16) || !aligned16(o_amax_partials) ||
+        (k_cache && (!aligned16(k_cache) || !aligned16(v_cache))))
+        return MQ_ERR_ALIGNMENT;
+    DeviceInfo *d = nullptr;
+    mq_status st = device_info(&d);
+    if (st != MQ_OK) return st;
+    const int grid = mq::attention_prefill_grid(M, H);
+    int slots = 0;   // one partial per CTA when they fit, else atomic max into zeroed slots
+    if (grid > MQ_AMAX_PARTIALS_MAX) {
+        slots = MQ_AMAX_PARTIALS_MAX;
+        if (cudaMemsetAsync(o_amax_partials, 0, sizeof(float) * MQ_AMAX_PARTIALS_MAX, stream) !=
+            cudaSuccess)
+            return MQ_ERR_CUDA;
+    }
+    *n_partials = slots ? slots : grid;
+    return cuda_status(mq::launch_attention_prefill(qkv_bf16, M, H, Hkv, k_cache, v_cache, S_max,
+                                                    o_bf16, o_amax_partials, slots, d->err, stream));
+}
+
+size_t mq_attention_decode_workspace_bytes(int64_t m, int64_t pos0, int64_t H, int64_t Hkv,
+                                           int64_t D) {
+    if (D != 128 || m < 1 || pos0 < 0 || H < 1 || Hkv < 1 || H % Hkv != 0) return 0;
+    return mq::attention_decode_workspace_bytes(m, pos0, H, Hkv);
+}
+
+mq_status mq_attention_decode_bf16(const void *qkv_bf16, int64_t m, int64_t pos0, int64_t H,
+                                   int64_t Hkv, int64_t D, void *k_cache, void *v_cache,
+                                   int64_t S_max, void *o_bf16, void *workspace, size_t ws_bytes,
+                                   cudaStream_t stream) {
+    if (!qkv_bf16 || !k_cache || !v_cache || !o_bf16 || !workspace) return MQ_ERR_INVALID_ARG;
+    if (D != 128 || H < 1 || Hkv < 1 || H % Hkv != 0 || m < 1 || pos0 < 0 ||
+        (H / Hkv) * m > mq::attention_decode_max_rows() || pos0 + m > S_max || S_max > (1LL << 24))
+        return MQ_ERR_SHAPE;
+    if (ws_bytes < mq::attention_decode_workspace_bytes(m, pos0, H, Hkv)) return MQ_ERR_INVALID_ARG;
+    if (!aligned16(qkv_bf16) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o_bf16) ||
+        !aligned16(workspace))
+        return MQ_ERR_ALIGNMENT;
+    DeviceInfo *d = nullptr;
+    mq_status st = device_info(&d);
+    if (st != MQ_OK) return st;
+    return cuda_status(mq::launch_attention_decode(qkv_bf16, m, pos0, H, Hkv, k_cache, v_cache,
+                                                   S_max, o_bf16, workspace, stream));
+}
+
 mq_status mq_decode_linear_bf16(const mq_weight *w, const void *x_bf16, int64_t M, void *y_bf16,
                                 cudaStream_t stream) {
     if (!x_bf16 || !y_bf16) return MQ_ERR_INVALID_ARG;

@@ -100,6 +100,23 @@ bool encode_codes_tmap(CUtensorMap *map, const void *codes, int64_t rows, int64_
 // 256-wide K step of one 128-row block.
 bool encode_sf_tmap(CUtensorMap *map, const void *sf, int64_t rows, int64_t K);
 
+// ---- attention (mq_attention.cu) ----------------------------------------------
+
+// CTAs of the prefill attention over M tokens and H query heads (head dim 128).
+int attention_prefill_grid(int64_t M, int64_t H);
+// Prefill attention; k_cache / v_cache NULL: no cache write.  partial_slots 0:
+// one amax partial per CTA; > 0: atomic max into that many (zeroed) slots.
+cudaError_t launch_attention_prefill(const void *qkv, int64_t M, int64_t H, int64_t Hkv,
+                                     void *k_cache, void *v_cache, int64_t S_max, void *o,
+                                     float *amax_partials, int partial_slots, unsigned *err,
+                                     cudaStream_t s);
+size_t attention_decode_workspace_bytes(int64_t m, int64_t pos0, int64_t H, int64_t Hkv);
+int attention_decode_max_rows();
+// Appends the m new tokens' K / V to the cache, then the decode attention.
+cudaError_t launch_attention_decode(const void *qkv, int64_t m, int64_t pos0, int64_t H, int64_t Hkv,
+                                    void *k_cache, void *v_cache, int64_t S_max, void *o, void *ws,
+                                    cudaStream_t s);
+
 // ---- decode (mq_decode.cu: BF16; mq_decode_nvf4.cu: NVFP4 W4A4) ----------------
 
 // Number of K slices the BF16 / NVFP4 (FP16-MMA) decode splits an [N, K]

@@ -107,6 +107,16 @@ __device__ __forceinline__ void tma_store_2d(const void *tmap, int32_t x, int32_
         : "memory");
 }
 
+// 3-D TMA tile store shared -> global (coordinates innermost first).
+__device__ __forceinline__ void tma_store_3d(const void *tmap, int32_t x, int32_t y, int32_t z,
+                                             uint32_t src) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+            reinterpret_cast<uint64_t>(tmap)),
+        "r"(x), "r"(y), "r"(z), "r"(src)
+        : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit_group() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -434,6 +444,60 @@ __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// 32 lanes x 32 consecutive 32-bit columns from registers: thread t of the
+// warp writes lane (warp's lane group base + t), columns [col, col+32).
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0],"
+        " {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16,"
+        " %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+        "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+        "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+// Waits until this thread's tcgen05.st writes have completed.
+__device__ __forceinline__ void tmem_st_wait() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// ---- tcgen05, single-CTA BF16 forms (kind::f16) -------------------------------------
+
+// D (TMEM, FP32) (+)= A * B, A and B BF16 from shared memory (descriptors),
+// M = 128, K = 16 per call.
+__device__ __forceinline__ void tc_mma_bf16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                               uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Same with A (M x K, BF16, one row per lane, two elements per 32-bit column)
+// read from tensor memory.
+__device__ __forceinline__ void tc_mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                               uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Instruction descriptor of kind::f16 with BF16 A and B and FP32 D: D format
+// 1 at bits [4,6), A / B format 1 (BF16) at [7,10) / [10,13), A / B major
+// (0 K-major, 1 MN-major) at bits 15 / 16, N >> 3 at [17,23), M >> 4 at [24,29).
+__host__ __device__ constexpr uint32_t idesc_bf16(uint32_t M, uint32_t N, uint32_t a_mn,
+                                                  uint32_t b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (a_mn << 15) | (b_mn << 16) | ((N >> 3) << 17) |
+           ((M >> 4) << 24);
+}
+
 // ---- shared-memory matrix descriptors (tcgen05) ---------------------------------
 // Fields: start address >> 4 in bits [0,14), leading byte offset >> 4 in
 // [16,30), stride byte offset >> 4 in [32,46), fixed version 1 at bit 46,
@@ -450,6 +514,20 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t saddr) {
     d |= static_cast<uint64_t>(1024u >> 4) << 32;    // SBO: 8 rows x 128 B
     d |= static_cast<uint64_t>(1u) << 46;            // version
     d |= static_cast<uint64_t>(2u) << 61;            // SWIZZLE_128B
+    return d;
+}
+
+// MN-major operand tile with 128-byte swizzle: 64 consecutive MN elements
+// (128 bytes) per K row, K rows 128 bytes apart, 8-row groups 1024 bytes apart
+// (SBO), the next 64 MN elements `mn_stride` bytes further (LBO) -- the TMA
+// SWIZZLE_128B image of [K rows, 64 elements] boxes placed mn_stride apart.
+__device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(uint32_t saddr, uint32_t mn_stride) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((mn_stride >> 4) & 0x3FFFu) << 16;   // LBO
+    d |= static_cast<uint64_t>(1024u >> 4) << 32;                   // SBO: 8 rows x 128 B
+    d |= static_cast<uint64_t>(1u) << 46;
+    d |= static_cast<uint64_t>(2u) << 61;                           // SWIZZLE_128B
     return d;
 }
 
