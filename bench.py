@@ -493,6 +493,159 @@ def measure_light(key, args, mq, dev, stream, flush, capture, replay_ms, pk):
     return r
 
 
+def measure_layer(args, mq, dev, stream, flush, capture, replay_ms, pk):
+    """A whole Llama-3-8B-shaped layer at 8192 tokens, NVFP4 prefill against
+    the same layer in BF16: RMSNorm -> QKV -> causal attention (32 query
+    heads, 8 KV heads, head dim 128; writes the BF16 KV cache) -> O ->
+    RMSNorm -> gate/up -> SwiGLU -> down.  NVFP4 path: this library's kernels
+    only (the RMSNorms and the attention emit the next quantizer's amax).
+    BF16 path: torch's rms_norm, cuBLAS matmuls, torch's scaled-dot-product
+    attention (flash / cuDNN) and a copy of K, V into the cache.  Also: each
+    attention alone, and the decode step's attention block (BF16 QKV ->
+    attention over the cache -> BF16 O) for 1 and 8 new tokens."""
+    M, H, Hkv, Dh, E, I = 8192, 32, 8, 128, 4096, 14336
+    Nqkv = (H + 2 * Hkv) * Dh
+    seed = 6
+    bf, u8, f32 = torch.bfloat16, torch.uint8, torch.float32
+    d = str(dev)
+    x = workloads.activation("channel_gain", M, E, seed, 0, device=d)
+    g1 = workloads.rmsnorm_gain(E, seed, 1, device=d)
+    g2 = workloads.rmsnorm_gain(E, seed, 2, device=d)
+    ws_ = [workloads.weight(n, k, 0.02, seed, 100 + i, device=d)
+           for i, (n, k) in enumerate([(Nqkv, E), (E, E), (2 * I, E), (E, I)])]
+    Wqkv, Wo, Wgu, Wd = [mq.Weight(w) for w in ws_]
+    S_max = M + 16
+    kc = torch.zeros(Hkv, S_max, Dh, dtype=bf, device=dev)
+    vc = torch.zeros_like(kc)
+    xn = torch.empty(M, E, dtype=bf, device=dev)
+    qkv = torch.empty(M, Nqkv, dtype=bf, device=dev)
+    o = torch.empty(M, E, dtype=bf, device=dev)
+    yo = torch.empty(M, E, dtype=bf, device=dev)
+    xn2 = torch.empty(M, E, dtype=bf, device=dev)
+    h = torch.empty(M, I, dtype=bf, device=dev)
+    y = torch.empty(M, E, dtype=bf, device=dev)
+
+    def qb(K):
+        return dict(codes=torch.empty(M, K // 2, dtype=u8, device=dev),
+                    sf=torch.empty(mq.mq_sf_bytes(M, K), dtype=u8, device=dev),
+                    s=torch.empty(1, dtype=f32, device=dev),
+                    part=torch.empty(mq.MQ_AMAX_PARTIALS_MAX, dtype=f32, device=dev))
+    q1, q2, q3, q4 = qb(E), qb(E), qb(E), qb(I)
+    st = {}
+
+    def attn():
+        st["n2"] = mq.mq_attention_prefill_bf16(qkv, M, H, Hkv, Dh, kc, vc, S_max, o, q2["part"], stream)
+
+    def nvfp4_layer():
+        st["n1"] = mq.mq_rmsnorm_amax(x, g1, RMS_EPS, M, E, E, xn, q1["part"], stream)
+        mq.mq_quantize_nvfp4(xn, M, E, E, q1["codes"], q1["sf"], q1["s"], amax_partials=q1["part"],
+                             n_partials=st["n1"], stream=stream)
+        mq.mq_gemm_nvfp4(q1["codes"], q1["sf"], q1["s"], M, Wqkv.handle, qkv, Nqkv, stream)
+        attn()
+        mq.mq_quantize_nvfp4(o, M, E, E, q2["codes"], q2["sf"], q2["s"], amax_partials=q2["part"],
+                             n_partials=st["n2"], stream=stream)
+        mq.mq_gemm_nvfp4(q2["codes"], q2["sf"], q2["s"], M, Wo.handle, yo, E, stream)
+        st["n3"] = mq.mq_rmsnorm_amax(yo, g2, RMS_EPS, M, E, E, xn2, q3["part"], stream)
+        mq.mq_quantize_nvfp4(xn2, M, E, E, q3["codes"], q3["sf"], q3["s"], amax_partials=q3["part"],
+                             n_partials=st["n3"], stream=stream)
+        st["n4"] = mq.mq_gemm_nvfp4_swiglu(q3["codes"], q3["sf"], q3["s"], M, Wgu.handle, h,
+                                           q4["part"], stream)
+        mq.mq_quantize_nvfp4(h, M, I, I, q4["codes"], q4["sf"], q4["s"], amax_partials=q4["part"],
+                             n_partials=st["n4"], stream=stream)
+        mq.mq_gemm_nvfp4(q4["codes"], q4["sf"], q4["s"], M, Wd.handle, y, E, stream)
+
+    def sdpa(t=None):
+        t = qkv if t is None else t
+        q = t[:, :H * Dh].view(M, H, Dh).transpose(0, 1)
+        k = t[:, H * Dh:(H + Hkv) * Dh].view(M, Hkv, Dh).transpose(0, 1)
+        v = t[:, (H + Hkv) * Dh:].view(M, Hkv, Dh).transpose(0, 1)
+        kc[:, :M].copy_(k)
+        vc[:, :M].copy_(v)
+        return torch.nn.functional.scaled_dot_product_attention(
+            q.unsqueeze(0), k.unsqueeze(0), v.unsqueeze(0), is_causal=True,
+            enable_gqa=True)[0].transpose(0, 1).reshape(M, H * Dh)
+
+    def bf16_layer():
+        a = torch.nn.functional.rms_norm(x, (E,), weight=g1, eps=RMS_EPS)
+        ob = sdpa(torch.matmul(a, ws_[0].t()))
+        yb = torch.matmul(ob, ws_[1].t())
+        a2 = torch.nn.functional.rms_norm(yb, (E,), weight=g2, eps=RMS_EPS)
+        gu = torch.matmul(a2, ws_[2].t())
+        hb = torch.nn.functional.silu(gu[:, :I]) * gu[:, I:]
+        torch.matmul(hb, ws_[3].t())
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def timed(fn, n):
+        fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(n):
+            flush()
+            a, b = ev(), ev()
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    n = max(3, args.config_steps)
+    t_nv = timed(nvfp4_layer, n)
+    if mq.mq_check(stream) != 0:
+        raise RuntimeError("device error in the layer")
+    t_attn = timed(attn, n)
+    t_sdpa = timed(sdpa, n)
+    t_bf = timed(bf16_layer, n)
+    attn_flops = 4.0 * Dh * H * M * (M + 1) / 2
+    lin_flops = 2.0 * M * E * (Nqkv + E + 2 * I) + 2.0 * M * I * E
+    r = {"workload": "llama3-8b layer (rmsnorm, qkv, causal gqa attention + kv cache, o, rmsnorm, "
+                     "swiglu mlp), 8192 tokens", "tokens": M, "heads": H, "kv_heads": Hkv,
+         "head_dim": Dh, "steps": n, "warmup": 1,
+         "prefill_layer_ms": round(t_nv, 4), "bf16_layer_ms": round(t_bf, 4),
+         "layer_speedup_vs_bf16": round(t_bf / t_nv, 3),
+         "layer_tflops": round((attn_flops + lin_flops) / (t_nv * 1e-3) / 1e12, 1),
+         "attention_ms": round(t_attn, 4),
+         "attention_tflops": round(attn_flops / (t_attn * 1e-3) / 1e12, 1),
+         "sdpa_ms": round(t_sdpa, 4),
+         "sdpa_tflops": round(attn_flops / (t_sdpa * 1e-3) / 1e12, 1),
+         "attention_flops": attn_flops, "linear_flops": lin_flops,
+         "note": "NVFP4 layer: this library's kernels only; BF16 layer: torch rms_norm, cuBLAS, "
+                 "torch SDPA (flash/cuDNN) + cache copy; sdpa_ms includes the K/V cache copy; "
+                 "L2 flushed before each timed layer; medians of event-timed runs"}
+    # decode step's attention block on the cache the prefill wrote: BF16 QKV
+    # -> attention over 8192 + m positions -> BF16 O (device time, graph replays)
+    R = 16
+    t_flush = replay_ms(capture([]))
+    dec = {}
+    for m in (1, 8):
+        xt = x[:m].contiguous()
+        qkv_t = torch.empty(m, Nqkv, dtype=bf, device=dev)
+        ot = torch.empty(m, E, dtype=bf, device=dev)
+        yt = torch.empty(m, E, dtype=bf, device=dev)
+        nbd = mq.mq_attention_decode_workspace_bytes(m, M, H, Hkv, Dh)
+        wsd = torch.empty(nbd, dtype=u8, device=dev)
+        body = [lambda s2, xt=xt, qkv_t=qkv_t, m=m: mq.mq_decode_linear_bf16(Wqkv.handle, xt, m, qkv_t, s2),
+                lambda s2, qkv_t=qkv_t, ot=ot, wsd=wsd, nbd=nbd, m=m: mq.mq_attention_decode_bf16(
+                    qkv_t, m, M, H, Hkv, Dh, kc, vc, S_max, ot, wsd, nbd, s2),
+                lambda s2, ot=ot, yt=yt, m=m: mq.mq_decode_linear_bf16(Wo.handle, ot, m, yt, s2)]
+        for f in body:
+            f(stream)
+        torch.cuda.synchronize()
+        g = capture(body)
+        dec[f"m{m}_ms"] = round((replay_ms(g) - t_flush) / R, 4)
+        del g
+    r["decode_attention_block"] = dec
+    r["decode_note"] = ("BF16 QKV decode linear -> decode attention over the 8192-token cache "
+                        "(appending the new tokens) -> BF16 O decode linear; device time per step "
+                        "from graph replays after an L2 flush")
+    if mq.mq_check(stream) != 0:
+        raise RuntimeError("device error in the layer decode")
+    for W in (Wqkv, Wo, Wgu, Wd):
+        W.free()
+    return r
+
+
 def run_gpu(args, wl, world, rank):
     from nvfp4_quantized_prefill_b200 import binding as mq
     mq.lib()
@@ -789,6 +942,9 @@ def run_gpu(args, wl, world, rank):
             per_config[key] = measure_light(key, args, mq, dev, stream, flush, capture,
                                             replay_ms, pk)
             torch.cuda.empty_cache()
+        per_config["llama3_8b_layer"] = measure_layer(args, mq, dev, stream, flush, capture,
+                                                      replay_ms, pk)
+        torch.cuda.empty_cache()
         if mq.mq_check(stream) != 0:
             raise RuntimeError("device error during the per-workload measurements")
 

@@ -16,8 +16,8 @@
 // first.  Warp 0 loads Q once and K / V tiles (TMA, 128-byte swizzle) into a
 // 2-stage ring; warp 1 issues S = Q K^T (kind::f16, M = 128, N = 128, K = 16
 // per instruction) into one of two 128-column FP32 buffers in tensor memory,
-// and O += P V with P read from tensor memory; warps 2-5 (one query row per
-// thread) take the row maximum, raise the running maximum only when it grows
+// and O += P V with P read from tensor memory; warps 2-9 (two threads per
+// query row, 64 columns each) take the row maximum, raise the running maximum only when it grows
 // by more than 2^8 (then O is rescaled in place; otherwise the stale maximum
 // keeps every weight below 2^8 and the final division by the same-based sum is
 // exact), write P as BF16 over the S buffer, and finally divide O by the row
@@ -43,10 +43,14 @@ constexpr uint32_t kQOff = 0;
 constexpr uint32_t kKOff = kTileBytes;                       // K stages
 constexpr uint32_t kVOff = kKOff + kStages * kTileBytes;     // V stages
 constexpr uint32_t kBarOff = kVOff + kStages * kTileBytes;
-constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;
-constexpr int kThreads = 192;             // producer, MMA, 4 softmax warps
-constexpr uint32_t kTmemCols = 512;       // S0 [0,128), S1 [128,256), O [256,384)
-constexpr uint32_t kOCol = 256;
+constexpr uint32_t kXchgOff = kBarOff + 256;                 // row maxima, 2 tiles x 2 halves x 128
+constexpr uint32_t kLsumOff = kXchgOff + 2 * 2 * 128 * 4;    // row sums, 2 halves x 128
+constexpr uint32_t kSmemBytes = kLsumOff + 2 * 128 * 4 + 1024;
+constexpr int kSoftmaxWarps = 8;          // two warpgroups: columns 0-63 and 64-127 of every row
+constexpr int kThreads = 32 * (2 + kSoftmaxWarps);   // producer, MMA, softmax
+constexpr int kSBufs = 3;                 // S / P buffers in tensor memory
+constexpr uint32_t kTmemCols = 512;       // S0, S1, S2 at 0, 128, 256; O at 384
+constexpr uint32_t kOCol = 128 * kSBufs;
 // log2(e) / sqrt(128): scores in the base-2 exponent domain
 constexpr float kScaleLog2 = 0.12751743082459868f;
 constexpr float kRescaleThreshold = 8.0f;  // raise the running max past 2^8 growth only
@@ -79,15 +83,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t s0 = smem_u32(smem);
     const uint32_t bar = s0 + kBarOff;
     const uint32_t q_full = bar;
-    const uint32_t k_full = bar + 8;          // [2]
+    const uint32_t k_full = bar + 8;          // [2] per K/V stage
     const uint32_t v_full = bar + 24;         // [2]
     const uint32_t kv_empty = bar + 40;       // [2]
-    const uint32_t s_full = bar + 56;         // [2]
-    const uint32_t p_full = bar + 72;         // [2]
-    const uint32_t o_done = bar + 88;
-    const uint32_t drain = bar + 96;          // every MMA issued has completed
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kBarOff + 112);
-    float *red = reinterpret_cast<float *>(smem + kBarOff + 128);   // 4 floats
+    const uint32_t s_full = bar + 56;         // [3] per S buffer
+    const uint32_t p_full = bar + 80;         // [3]
+    const uint32_t pv_done = bar + 104;       // [3] the PV product that read P of that buffer
+    const uint32_t drain = bar + 128;         // every MMA issued has completed
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kBarOff + 136);
+    float *red = reinterpret_cast<float *>(smem + kBarOff + 160);   // 8 floats
+    float *xchg = reinterpret_cast<float *>(smem + kXchgOff);      // [2][2][128]
+    float *lsum = reinterpret_cast<float *>(smem + kLsumOff);      // [2][128]
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -106,10 +112,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(k_full + 8 * i, 1);
             mbar_init(v_full + 8 * i, 1);
             mbar_init(kv_empty + 8 * i, 1);
-            mbar_init(s_full + 8 * i, 1);
-            mbar_init(p_full + 8 * i, 4);     // one arrival per softmax warp
         }
-        mbar_init(o_done, 1);
+        for (int i = 0; i < kSBufs; ++i) {
+            mbar_init(s_full + 8 * i, 1);
+            mbar_init(p_full + 8 * i, kSoftmaxWarps);   // one arrival per softmax warp
+            mbar_init(pv_done + 8 * i, 1);
+        }
         mbar_init(drain, 1);
         fence_barrier_init();
         prefetch_tmap(&tmap_qkv);
@@ -184,35 +192,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             for (int j = 0; j <= nkv && ok; ++j) {
                 if (j < nkv) {
-                    const int st = j & 1;
+                    const int st = j & 1, sb = j % kSBufs;
                     if (!wait_bar(k_full + 8 * st, (j >> 1) & 1)) ok = false;
-                    // S buffer st last held P_{j-2}: its PV must have completed
-                    if (j >= 2 && !wait_bar(o_done, (j - 2) & 1)) ok = false;
+                    // S buffer sb last held P_{j-3}: its PV must have completed
+                    if (j >= kSBufs && !wait_bar(pv_done + 8 * sb, ((j - kSBufs) / kSBufs) & 1)) ok = false;
                     tc_fence_after();
-                    const uint32_t ks = s0 + kKOff + st * kTileBytes;
-#pragma unroll
-                    for (int kk = 0; kk < kD / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32u;
-                        tc_mma_bf16_ss(tmem + st * 128u, sdesc_kmajor_sw128(s0 + kQOff + off),
-                                       sdesc_kmajor_sw128(ks + off), idesc_s, kk > 0 ? 1u : 0u);
-                    }
-                    tc_commit(s_full + 8 * st);
+                    tc_mma8_bf16_ss_commit(tmem + sb * 128u, sdesc_kmajor_sw128(s0 + kQOff),
+                                           sdesc_kmajor_sw128(s0 + kKOff + st * kTileBytes), idesc_s, 0u,
+                                           s_full + 8 * sb);
                 }
                 if (j >= 1) {
-                    const int jj = j - 1, st = jj & 1;
-                    if (!wait_bar(p_full + 8 * st, (jj >> 1) & 1)) ok = false;
+                    const int jj = j - 1, st = jj & 1, sb = jj % kSBufs;
+                    if (!wait_bar(p_full + 8 * sb, (jj / kSBufs) & 1)) ok = false;
                     if (!wait_bar(v_full + 8 * st, (jj >> 1) & 1)) ok = false;
                     tc_fence_after();
-                    const uint32_t vs = s0 + kVOff + st * kTileBytes;
-#pragma unroll
-                    for (int kk = 0; kk < kTile / 16; ++kk) {
-                        // keys 16 kk .. 16 kk + 15: two 8-row groups of the V tile
-                        tc_mma_bf16_ts(tmem + kOCol, tmem + st * 128u + kk * 8u,
-                                       sdesc_mnmajor_sw128(vs + kk * 2048u, kHalfBytes), idesc_o,
-                                       (jj > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    tc_commit(o_done);
-                    tc_commit(kv_empty + 8 * st);
+                    // keys 16 kk .. 16 kk + 15: two 8-row groups of the V tile
+                    tc_mma8_bf16_ts_commit2(tmem + kOCol, tmem + sb * 128u,
+                                            sdesc_mnmajor_sw128(s0 + kVOff + st * kTileBytes, kHalfBytes),
+                                            idesc_o, jj > 0 ? 1u : 0u, pv_done + 8 * sb,
+                                            kv_empty + 8 * st);
                 }
             }
             // every MMA this thread issued completes before TMEM is freed
@@ -222,77 +220,112 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else {
         // ---------------------------------------------------------- softmax
+        // warpgroup wg holds columns [64 wg, 64 wg + 64) of every row; the two
+        // threads of a row agree on the row maximum through shared memory
+        // (one named barrier a tile, double-buffered by tile parity) and keep
+        // their own share of the row sum
+        const int wg = (warp - 2) >> 2;
         const int quarter = warp & 3;             // TMEM lane group of this warp
         const int r = quarter * 32 + lane;        // query row in the tile
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        const int col0 = wg * 64;
         float m_run = -INFINITY, l = 0.0f;
-        for (int j = 0; j < nkv && ok; ++j) {
-            const int st = j & 1;
-            ok = __all_sync(0xFFFFFFFFu, wait_bar(s_full + 8 * st, (j >> 1) & 1)) && ok;
+        for (int j = 0; j < nkv; ++j) {
+            const int st = j & 1, sb = j % kSBufs;
+            ok = __all_sync(0xFFFFFFFFu, wait_bar(s_full + 8 * sb, (j / kSBufs) & 1)) && ok;
             tc_fence_after();
-            uint32_t sr[kTile];
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                tmem_ld32(tmem + lane_off + st * 128u + c * 32u, *reinterpret_cast<uint32_t (*)[32]>(&sr[c * 32]));
+            uint32_t sr[64];
+            tmem_ld32(tmem + lane_off + sb * 128u + col0, *reinterpret_cast<uint32_t (*)[32]>(&sr[0]));
+            tmem_ld32(tmem + lane_off + sb * 128u + col0 + 32u, *reinterpret_cast<uint32_t (*)[32]>(&sr[32]));
             tmem_ld_wait();
-            float s[kTile];
-            float mx = -INFINITY;
+            float s[64];
+            float mp[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mp[e] = -INFINITY;
             const bool diag = (j == qt);
 #pragma unroll
-            for (int c = 0; c < kTile; ++c) {
+            for (int c = 0; c < 64; ++c) {
                 float x = __uint_as_float(sr[c]) * kScaleLog2;
-                if (diag && c > r) x = -INFINITY;
+                if (diag && col0 + c > r) x = -INFINITY;
                 s[c] = x;
-                mx = fmaxf(mx, x);
+                mp[c & 7] = fmaxf(mp[c & 7], x);   // eight independent chains
             }
+            float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+            xchg[(st * 2 + wg) * 128 + r] = mx;
+            // the barrier's AND also carries "every softmax warp saw S": after
+            // a timed-out wait all eight warps leave the loop together (none
+            // may be left waiting here for the others)
+            uint32_t all_ok;
+            asm volatile(
+                "{\n\t.reg .pred p, q;\n\t"
+                "setp.ne.u32 p, %1, 0;\n\t"
+                "bar.red.and.pred q, 2, 256, p;\n\t"
+                "selp.u32 %0, 1, 0, q;\n\t}"
+                : "=r"(all_ok)
+                : "r"(ok ? 1u : 0u)
+                : "memory");
+            if (!all_ok) {
+                ok = false;
+                break;
+            }
+            mx = fmaxf(mx, xchg[(st * 2 + (1 - wg)) * 128 + r]);
             // raise the running maximum only for a growth beyond 2^8 (or at
             // the first tile); O then needs the factor 2^(m_old - m_new)
             const bool need = mx > m_run + kRescaleThreshold;
             const float m_new = need ? mx : m_run;
             const float f = need ? exp2f(m_run - m_new) : 1.0f;   // 0 at the first tile
             if (__any_sync(0xFFFFFFFFu, need) && j > 0) {
-                ok = __all_sync(0xFFFFFFFFu, wait_bar(o_done, (j - 1) & 1)) && ok;
+                // (a timeout here is seen by the other warps at the next
+                // tile's barrier)
+                ok = __all_sync(0xFFFFFFFFu,
+                                wait_bar(pv_done + 8 * ((j - 1) % kSBufs), ((j - 1) / kSBufs) & 1)) && ok;
                 tc_fence_after();
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < 2; ++c) {
                     uint32_t ov[32];
-                    tmem_ld32(tmem + lane_off + kOCol + c * 32u, ov);
+                    tmem_ld32(tmem + lane_off + kOCol + col0 + c * 32u, ov);
                     tmem_ld_wait();
 #pragma unroll
                     for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
-                    tmem_st32(tmem + lane_off + kOCol + c * 32u, ov);
+                    tmem_st32(tmem + lane_off + kOCol + col0 + c * 32u, ov);
                 }
                 tmem_st_wait();
             }
             l *= f;
             m_run = m_new;
-            uint32_t pk[kTile / 2];
+            uint32_t pk[32];
+            float lp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-            for (int c = 0; c < kTile / 2; ++c) {
+            for (int c = 0; c < 32; ++c) {
                 const __nv_bfloat162 pb =
                     __floats2bfloat162_rn(exp2f(s[2 * c] - m_run), exp2f(s[2 * c + 1] - m_run));
                 // the row sum of the BF16 weights the PV product uses
-                l += __bfloat162float(pb.x) + __bfloat162float(pb.y);
+                lp[c & 3] += __bfloat162float(pb.x) + __bfloat162float(pb.y);
                 pk[c] = *reinterpret_cast<const uint32_t *>(&pb);
             }
-            tmem_st32(tmem + lane_off + st * 128u, *reinterpret_cast<uint32_t (*)[32]>(&pk[0]));
-            tmem_st32(tmem + lane_off + st * 128u + 32u, *reinterpret_cast<uint32_t (*)[32]>(&pk[32]));
+            l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
+            tmem_st32(tmem + lane_off + sb * 128u + wg * 32u, pk);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full + 8 * st);
+            if (lane == 0) mbar_arrive(p_full + 8 * sb);
         }
-        // epilogue: O / l -> BF16, and max |o| of the tile
-        ok = __all_sync(0xFFFFFFFFu, wait_bar(o_done, (nkv - 1) & 1)) && ok;
+        // epilogue: O / l -> BF16 (this half's 64 columns), and max |o|
+        lsum[wg * 128 + r] = l;
+        asm volatile("bar.sync 3, 256;" ::: "memory");
+        l += lsum[(1 - wg) * 128 + r];
+        ok = __all_sync(0xFFFFFFFFu,
+                        wait_bar(pv_done + 8 * ((nkv - 1) % kSBufs), ((nkv - 1) / kSBufs) & 1)) && ok;
         tc_fence_after();
         const float inv = 1.0f / l;
         const int row = qt * kTile + r;
         float omax = 0.0f;
-        __nv_bfloat16 *orow = p.o + static_cast<int64_t>(row) * (p.H * kD) + h * kD;
+        __nv_bfloat16 *orow = p.o + static_cast<int64_t>(row) * (p.H * kD) + h * kD + col0;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
             uint32_t ov[32];
-            tmem_ld32(tmem + lane_off + kOCol + c * 32u, ov);
+            tmem_ld32(tmem + lane_off + kOCol + col0 + c * 32u, ov);
             tmem_ld_wait();
             uint32_t pk[16];
 #pragma unroll
@@ -312,9 +345,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (row >= p.M) omax = 0.0f;
         const uint32_t b = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(omax));
         if (lane == 0) red[warp - 2] = __uint_as_float(b);
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        asm volatile("bar.sync 1, 256;" ::: "memory");
         if (warp == 2 && lane == 0) {
-            const float m = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+            float m = 0.0f;
+            for (int i = 0; i < kSoftmaxWarps; ++i) m = fmaxf(m, red[i]);
             if (p.partial_slots > 0)
                 atomicMax(reinterpret_cast<unsigned *>(p.amax_partials) + blockIdx.x % p.partial_slots,
                           __float_as_uint(m));   // non-negative floats order like their bits
@@ -358,12 +392,19 @@ EncodeFn encode_fn() {
 // unnormalised o) per query row, and a combine pass merges the chunks.
 // FP32 throughout (scores, weights, accumulation); BF16 output.
 
-constexpr int kDecChunk = 128;            // keys per CTA
+constexpr int kDecChunk = 128;            // keys per sub-chunk in shared memory
+// 128-key sub-chunks per CTA: four (512 keys) for up to 8 query rows, where a
+// CTA's work is mostly the cache read; one for more rows, where the FP32
+// arithmetic per key grows and more CTAs share it
+__host__ __device__ constexpr int dec_sub(int64_t rows) { return rows <= 8 ? 4 : 1; }
 constexpr int kDecThreads = 256;
 constexpr int kDecMaxRows = 64;           // query rows per KV head (group size x tokens)
 constexpr int kKPad = kD + 2;             // padded K row in shared memory (conflict-free dot products)
-constexpr uint32_t kDecSmem = kDecChunk * kKPad * 2 + kDecChunk * kD * 2 +
-                              kDecMaxRows * kD * 4 + kDecMaxRows * kDecChunk * 4;
+// shared memory: the chunk's K (padded rows) and V, then per query row its
+// FP32 query and its chunk of scores / weights (sized by the row count, so
+// that a one-token step fits three CTAs on an SM)
+constexpr uint32_t kDecSmemFixed = kDecChunk * kKPad * 2 + kDecChunk * kD * 2;
+constexpr uint32_t kDecSmemPerRow = kD * 4 + kDecChunk * 4;
 
 struct DecodeParams {
     const __nv_bfloat16 *qkv;   // [m, (H + 2 Hkv) * 128]
@@ -372,6 +413,7 @@ struct DecodeParams {
     __nv_bfloat16 *o;           // [m, H * 128]
     float *part;                // [Hkv, n_chunks, rows, 2 + 128]
     int m, pos0, H, Hkv, S_max, n_chunks, rows;
+    int n_sub;                  // 128-key sub-chunks per CTA
 };
 
 // Copies the new tokens' K and V rows into the cache (grid m x Hkv, 32 threads).
@@ -391,105 +433,146 @@ __global__ void __launch_bounds__(32) kv_append_kernel(const DecodeParams p) {
         reinterpret_cast<uint4 *>(p.v_cache + dst)[lane - 16] = src_v[lane - 16];
 }
 
-__global__ void __launch_bounds__(kDecThreads) attention_decode_kernel(const DecodeParams p) {
+// kRows: the largest query-row count this instance serves (its share of o in
+// registers scales with it)
+template <int kRows>
+__global__ void __launch_bounds__(kDecThreads, 2) attention_decode_kernel(const DecodeParams p) {
     extern __shared__ __align__(16) uint8_t dsm[];
     __nv_bfloat16 *ks = reinterpret_cast<__nv_bfloat16 *>(dsm);                       // [128][130]
     __nv_bfloat16 *vs = ks + kDecChunk * kKPad;                                          // [128][128]
     float *qs = reinterpret_cast<float *>(vs + kDecChunk * kD);                          // [rows][128]
-    float *ss = qs + kDecMaxRows * kD;                                                   // [rows][128]
+    float *ss = qs + p.rows * kD;                                                        // [rows][128]
+    __shared__ float m_run[kDecMaxRows], l_run[kDecMaxRows], alpha[kDecMaxRows];
     const int c = blockIdx.x, g = blockIdx.y, tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
     const int group = p.H / p.Hkv;
     const int n_keys = p.pos0 + p.m;
-    const int key0 = c * kDecChunk;
-    const int nk = min(kDecChunk, n_keys - key0);
     const int cols = (p.H + 2 * p.Hkv) * kD;
     griddep_wait();            // the appended rows and the queries are in place
     griddep_launch_dependents();
-    // the chunk's keys and values (rows past the chunk read as zero)
-    for (int i = tid; i < kDecChunk * (kD / 8); i += kDecThreads) {
-        const int k = i / (kD / 8), d8 = (i % (kD / 8)) * 8;
-        uint4 kv = make_uint4(0, 0, 0, 0), vv = kv;
-        if (k < nk) {
-            const int64_t off = (static_cast<int64_t>(g) * p.S_max + key0 + k) * kD + d8;
-            kv = *reinterpret_cast<const uint4 *>(p.k_cache + off);
-            vv = *reinterpret_cast<const uint4 *>(p.v_cache + off);
-        }
-        const uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e)   // the padded K rows are only 4-byte aligned
-            *reinterpret_cast<uint32_t *>(ks + k * kKPad + d8 + 2 * e) = w[e];
-        *reinterpret_cast<uint4 *>(vs + k * kD + d8) = vv;
-    }
     // the group's query rows: row rr = hh * m + t (head g * group + hh, token t)
     for (int i = tid; i < p.rows * kD; i += kDecThreads) {
         const int rr = i / kD, d = i % kD, hh = rr / p.m, t = rr % p.m;
         qs[rr * kD + d] = __bfloat162float(p.qkv[static_cast<int64_t>(t) * cols + (g * group + hh) * kD + d]);
     }
-    __syncthreads();
-    // scores: thread -> one key, every other row
-    {
-        const int k = tid & (kDecChunk - 1), half = tid >> 7;
-        float kr[kD];
+    for (int rr = tid; rr < p.rows; rr += kDecThreads) {
+        m_run[rr] = -INFINITY;
+        l_run[rr] = 0.0f;
+    }
+    // this thread's share of o: dimension d of rows half, half + 2, ...
+    const int d = tid & (kD - 1), half = tid >> 7;
+    float acc[kRows / 2];
 #pragma unroll
-        for (int d = 0; d < kD; d += 2) {
-            const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(ks + k * kKPad + d);
-            kr[d] = __bfloat162float(b.x);
-            kr[d + 1] = __bfloat162float(b.y);
-        }
-        const int pos = key0 + k;
-        for (int rr = half; rr < p.rows; rr += 2) {
-            const float *q = qs + rr * kD;
-            float acc = 0.0f;
-#pragma unroll
-            for (int d = 0; d < kD; d += 4) {
-                const float4 qv = *reinterpret_cast<const float4 *>(q + d);
-                acc = fmaf(qv.x, kr[d], acc);
-                acc = fmaf(qv.y, kr[d + 1], acc);
-                acc = fmaf(qv.z, kr[d + 2], acc);
-                acc = fmaf(qv.w, kr[d + 3], acc);
+    for (int i = 0; i < kRows / 2; ++i) acc[i] = 0.0f;
+    // the CTA's keys: n_sub 128-key sub-chunks, merged on the fly
+    for (int sc = 0; sc < p.n_sub; ++sc) {
+        const int key0 = (c * p.n_sub + sc) * kDecChunk;
+        const int nk = min(kDecChunk, n_keys - key0);
+        if (nk <= 0) break;    // uniform over the CTA
+        __syncthreads();       // the previous sub-chunk's K, V and weights are consumed
+        for (int i = tid; i < kDecChunk * (kD / 8); i += kDecThreads) {
+            const int k = i / (kD / 8), d8 = (i % (kD / 8)) * 8;
+            uint4 kv = make_uint4(0, 0, 0, 0), vv = kv;
+            if (k < nk) {
+                const int64_t off = (static_cast<int64_t>(g) * p.S_max + key0 + k) * kD + d8;
+                kv = *reinterpret_cast<const uint4 *>(p.k_cache + off);
+                vv = *reinterpret_cast<const uint4 *>(p.v_cache + off);
             }
-            const int t = rr % p.m;
-            ss[rr * kDecChunk + k] = (k < nk && pos <= p.pos0 + t) ? acc * kScaleLog2 : -INFINITY;
+            const uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)   // the padded K rows are only 4-byte aligned
+                *reinterpret_cast<uint32_t *>(ks + k * kKPad + d8 + 2 * e) = w[e];
+            *reinterpret_cast<uint4 *>(vs + k * kD + d8) = vv;
+        }
+        __syncthreads();
+        // scores: thread -> one key, every other row
+        {
+            const int k = tid & (kDecChunk - 1);
+            uint32_t kr[kD / 2];   // the key's 128 values, two BF16 a register
+#pragma unroll
+            for (int dd = 0; dd < kD; dd += 2) kr[dd / 2] = *reinterpret_cast<const uint32_t *>(ks + k * kKPad + dd);
+            const int pos = key0 + k;
+            for (int rr = half; rr < p.rows; rr += 2) {
+                const float *q = qs + rr * kD;
+                float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll
+                for (int dd = 0; dd < kD; dd += 4) {
+                    const float4 qv = *reinterpret_cast<const float4 *>(q + dd);
+                    a0 = fmaf(qv.x, __uint_as_float(kr[dd / 2] << 16), a0);
+                    a1 = fmaf(qv.y, __uint_as_float(kr[dd / 2] & 0xFFFF0000u), a1);
+                    a0 = fmaf(qv.z, __uint_as_float(kr[dd / 2 + 1] << 16), a0);
+                    a1 = fmaf(qv.w, __uint_as_float(kr[dd / 2 + 1] & 0xFFFF0000u), a1);
+                }
+                const int t = rr % p.m;
+                ss[rr * kDecChunk + k] = (k < nk && pos <= p.pos0 + t) ? (a0 + a1) * kScaleLog2 : -INFINITY;
+            }
+        }
+        __syncthreads();
+        // per row: running maximum, weights 2^(x - max), running sum (a warp a row)
+        for (int rr = warp; rr < p.rows; rr += kDecThreads / 32) {
+            float x[4], mx = -INFINITY;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                x[e] = ss[rr * kDecChunk + lane + 32 * e];
+                mx = fmaxf(mx, x[e]);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+            const float m_old = m_run[rr];
+            const float m_new = fmaxf(m_old, mx);
+            float sum = 0.0f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float w = m_new == -INFINITY ? 0.0f : exp2f(x[e] - m_new);
+                ss[rr * kDecChunk + lane + 32 * e] = w;
+                sum += w;
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+            __syncwarp();
+            if (lane == 0) {
+                const float a = (m_old == -INFINITY) ? 0.0f : exp2f(m_old - m_new);
+                alpha[rr] = a;
+                l_run[rr] = l_run[rr] * a + sum;
+                m_run[rr] = m_new;
+            }
+        }
+        __syncthreads();
+        // o: rescale, then add this sub-chunk's weighted values -- each value
+        // loaded once for all of this thread's rows (weights are broadcast)
+#pragma unroll
+        for (int i = 0; i < kRows / 2; ++i)
+            if (half + 2 * i < p.rows) acc[i] *= alpha[half + 2 * i];
+        for (int k = 0; k < nk; ++k) {
+            const float v = __bfloat162float(vs[k * kD + d]);
+#pragma unroll
+            for (int i = 0; i < kRows / 2; ++i) {
+                const int rr = half + 2 * i;
+                if (rr < p.rows) acc[i] = fmaf(ss[rr * kDecChunk + k], v, acc[i]);
+            }
         }
     }
     __syncthreads();
-    // per row: chunk max, weights 2^(x - max), their sum (a warp per row)
-    const int warp = tid >> 5, lane = tid & 31;
     float *part = p.part + (static_cast<int64_t>(g) * p.n_chunks + c) * p.rows * (2 + kD);
-    for (int rr = warp; rr < p.rows; rr += kDecThreads / 32) {
-        float x[4], mx = -INFINITY;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            x[e] = ss[rr * kDecChunk + lane + 32 * e];
-            mx = fmaxf(mx, x[e]);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-        float sum = 0.0f;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float w = mx == -INFINITY ? 0.0f : exp2f(x[e] - mx);
-            ss[rr * kDecChunk + lane + 32 * e] = w;
-            sum += w;
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
-        if (lane == 0) {
-            part[rr * (2 + kD)] = mx;
-            part[rr * (2 + kD) + 1] = sum;
-        }
+    for (int rr = tid; rr < p.rows; rr += kDecThreads) {
+        part[rr * (2 + kD)] = m_run[rr];
+        part[rr * (2 + kD) + 1] = l_run[rr];
     }
-    __syncthreads();
-    // unnormalised o: thread -> one dimension, every other row
-    {
-        const int d = tid & (kD - 1), half = tid >> 7;
-        for (int rr = half; rr < p.rows; rr += 2) {
-            const float *w = ss + rr * kDecChunk;
-            float acc = 0.0f;
-            for (int k = 0; k < nk; ++k) acc = fmaf(w[k], __bfloat162float(vs[k * kD + d]), acc);
-            part[rr * (2 + kD) + 2 + d] = acc;
-        }
+#pragma unroll
+    for (int i = 0; i < kRows / 2; ++i) {
+        const int rr = half + 2 * i;
+        if (rr < p.rows) part[rr * (2 + kD) + 2 + d] = acc[i];
     }
+}
+
+template <int kRows>
+cudaError_t launch_decode_rows(const DecodeParams &p, uint32_t smem, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(attention_decode_kernel<kRows>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kDecSmemFixed + kDecSmemPerRow * kRows);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(attention_decode_kernel<kRows>, dim3(p.n_chunks, p.Hkv), dim3(kDecThreads), smem,
+                      s, p);
 }
 
 // Merges the chunks of one query row (a CTA of 128 threads, one per dimension).
@@ -501,12 +584,14 @@ __global__ void __launch_bounds__(kD) attention_combine_kernel(const DecodeParam
     const float *base = p.part + static_cast<int64_t>(g) * p.n_chunks * p.rows * (2 + kD) + rr * (2 + kD);
     const int64_t step = static_cast<int64_t>(p.rows) * (2 + kD);
     float mx = -INFINITY;
+#pragma unroll 8
     for (int c = 0; c < p.n_chunks; ++c) mx = fmaxf(mx, base[c * step]);
     float l = 0.0f, acc = 0.0f;
+#pragma unroll 8
     for (int c = 0; c < p.n_chunks; ++c) {
         const float mc = base[c * step];
-        if (mc == -INFINITY) continue;   // no visible key in this chunk
-        const float f = exp2f(mc - mx);
+        // a chunk with no visible key (maximum -inf) adds nothing
+        const float f = mc == -INFINITY ? 0.0f : exp2f(mc - mx);
         l = fmaf(base[c * step + 1], f, l);
         acc = fmaf(base[c * step + 2 + d], f, acc);
     }
@@ -516,8 +601,9 @@ __global__ void __launch_bounds__(kD) attention_combine_kernel(const DecodeParam
 }  // namespace
 
 size_t attention_decode_workspace_bytes(int64_t m, int64_t pos0, int64_t H, int64_t Hkv) {
-    const int64_t n_chunks = (pos0 + m + kDecChunk - 1) / kDecChunk;
     const int64_t rows = H / Hkv * m;
+    const int64_t span = kDecChunk * dec_sub(rows);
+    const int64_t n_chunks = (pos0 + m + span - 1) / span;
     return static_cast<size_t>(Hkv * n_chunks * rows * (2 + kD)) * sizeof(float);
 }
 
@@ -537,14 +623,14 @@ cudaError_t launch_attention_decode(const void *qkv, int64_t m, int64_t pos0, in
     p.H = static_cast<int>(H);
     p.Hkv = static_cast<int>(Hkv);
     p.S_max = static_cast<int>(S_max);
-    p.n_chunks = static_cast<int>((pos0 + m + kDecChunk - 1) / kDecChunk);
     p.rows = static_cast<int>(H / Hkv * m);
+    p.n_sub = dec_sub(p.rows);
+    p.n_chunks = static_cast<int>((pos0 + m + kDecChunk * p.n_sub - 1) / (kDecChunk * p.n_sub));
     cudaError_t e = launch_pdl(kv_append_kernel, dim3(p.m, p.Hkv), dim3(32), 0, s, p);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(attention_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kDecSmem);
-    if (e != cudaSuccess) return e;
-    e = launch_pdl(attention_decode_kernel, dim3(p.n_chunks, p.Hkv), dim3(kDecThreads), kDecSmem, s, p);
+    const uint32_t smem = kDecSmemFixed + kDecSmemPerRow * static_cast<uint32_t>(p.rows);
+    e = p.rows <= 8 ? launch_decode_rows<8>(p, smem, s)
+                    : (p.rows <= 32 ? launch_decode_rows<32>(p, smem, s) : launch_decode_rows<kDecMaxRows>(p, smem, s));
     if (e != cudaSuccess) return e;
     e = launch_pdl(attention_combine_kernel, dim3(p.rows, p.Hkv), dim3(kD), 0, s, p);
     return e != cudaSuccess ? e : cudaGetLastError();

@@ -489,6 +489,67 @@ __device__ __forceinline__ void tc_mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem,
         : "memory");
 }
 
+// Eight chained BF16 MMAs (K = 8 x 16) and a commit, from one issue block:
+// A and B from shared memory, K-major with 128-byte swizzle, the K steps 32
+// bytes apart inside a 64-element atom and `atom_bytes` apart across the two
+// atoms; the first MMA overwrites D when `accumulate` is 0.
+__device__ __forceinline__ void tc_mma8_bf16_ss_commit(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                       uint32_t idesc, uint32_t accumulate,
+                                                       uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .pred p, t;\n\t"
+        ".reg .b64 a1, a2, a3, a4, a5, a6, a7, b1, b2, b3, b4, b5, b6, b7;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\tsetp.eq.b32 t, 0, 0;\n\t"
+        "add.s64 a1, %1, 2;\n\tadd.s64 a2, %1, 4;\n\tadd.s64 a3, %1, 6;\n\t"
+        "add.s64 a4, %1, 1024;\n\tadd.s64 a5, %1, 1026;\n\tadd.s64 a6, %1, 1028;\n\t"
+        "add.s64 a7, %1, 1030;\n\t"
+        "add.s64 b1, %2, 2;\n\tadd.s64 b2, %2, 4;\n\tadd.s64 b3, %2, 6;\n\t"
+        "add.s64 b4, %2, 1024;\n\tadd.s64 b5, %2, 1026;\n\tadd.s64 b6, %2, 1028;\n\t"
+        "add.s64 b7, %2, 1030;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a2, b2, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a3, b3, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a4, b4, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a5, b5, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a6, b6, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a7, b7, %3, t;\n\t"
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%5];\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(bar)
+        : "memory");
+}
+
+// Eight chained BF16 MMAs with A from tensor memory (8 columns per K = 16
+// step) and B an MN-major shared-memory operand whose K steps are 2048 bytes
+// apart (two 8-row groups), then two commits.
+__device__ __forceinline__ void tc_mma8_bf16_ts_commit2(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                                        uint32_t idesc, uint32_t accumulate,
+                                                        uint32_t bar0, uint32_t bar1) {
+    asm volatile(
+        "{\n\t.reg .pred p, t;\n\t"
+        ".reg .b32 a1, a2, a3, a4, a5, a6, a7;\n\t"
+        ".reg .b64 b1, b2, b3, b4, b5, b6, b7;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\tsetp.eq.b32 t, 0, 0;\n\t"
+        "add.u32 a1, %1, 8;\n\tadd.u32 a2, %1, 16;\n\tadd.u32 a3, %1, 24;\n\t"
+        "add.u32 a4, %1, 32;\n\tadd.u32 a5, %1, 40;\n\tadd.u32 a6, %1, 48;\n\t"
+        "add.u32 a7, %1, 56;\n\t"
+        "add.s64 b1, %2, 128;\n\tadd.s64 b2, %2, 256;\n\tadd.s64 b3, %2, 384;\n\t"
+        "add.s64 b4, %2, 512;\n\tadd.s64 b5, %2, 640;\n\tadd.s64 b6, %2, 768;\n\t"
+        "add.s64 b7, %2, 896;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b2, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], b3, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a4], b4, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a5], b5, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a6], b6, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a7], b7, %3, t;\n\t"
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%5];\n\t"
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%6];\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(bar0), "r"(bar1)
+        : "memory");
+}
+
 // Instruction descriptor of kind::f16 with BF16 A and B and FP32 D: D format
 // 1 at bits [4,6), A / B format 1 (BF16) at [7,10) / [10,13), A / B major
 // (0 K-major, 1 MN-major) at bits 15 / 16, N >> 3 at [17,23), M >> 4 at [24,29).
