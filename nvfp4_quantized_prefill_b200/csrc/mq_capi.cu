@@ -15,6 +15,7 @@
 #include <mutex>
 
 #include "mq.h"
+#include "mq_debug.h"
 #include "mq_internal.h"
 
 // Per-device word in which kernels latch asynchronous errors (bounded waits
@@ -432,6 +433,46 @@ mq_status mq_gemm_nvfp4(const uint8_t *a_codes, const uint8_t *a_sf_swizzled,
     if (st != MQ_OK) return st;
     return gemm_impl(d, a_codes, a_sf_swizzled, a_s_enc_dev, M, w, y_bf16, ldy, false, nullptr,
                      nullptr, stream);
+}
+
+// Test-only entry point (include/mq_debug.h): the GEMM with every bounded
+// wait limited to wait_limit_us and the first K stage of the first tile never
+// released, so that the kernel's abort path runs: the producers' waits run out,
+// the timeout bit is latched, every role stops, drains what it issued and the
+// pair exits.  Not part of the public interface.
+mq_status mq_debug_gemm_withhold_release(const uint8_t *a_codes, const uint8_t *a_sf_swizzled,
+                                         const float *a_s_enc_dev, int64_t M, const mq_weight *w,
+                                         void *y_bf16, int64_t ldy, uint32_t wait_limit_us,
+                                         cudaStream_t stream) {
+    if (!a_codes || !a_sf_swizzled || !a_s_enc_dev || !y_bf16) return MQ_ERR_INVALID_ARG;
+    if (wait_limit_us < 1000 || wait_limit_us > 2000000u) return MQ_ERR_INVALID_ARG;
+    mq_status st = check_weight(w);
+    if (st != MQ_OK) return st;
+    // at least one tile and more K steps than ring stages (the withheld
+    // stage is waited for on the ring's second lap)
+    if (M < 1 || ldy < w->N || !shape_fits(M, w->K) || w->K < 2048) return MQ_ERR_SHAPE;
+    if (!aligned16(a_codes) || !aligned16(a_sf_swizzled) || !aligned16(y_bf16))
+        return MQ_ERR_ALIGNMENT;
+    DeviceInfo *d = nullptr;
+    st = device_info(&d);
+    if (st != MQ_OK) return st;
+    CUtensorMap ta, tsa;
+    if (!mq::encode_codes_tmap(&ta, a_codes, M, w->K)) return MQ_ERR_CUDA;
+    if (!mq::encode_sf_tmap(&tsa, a_sf_swizzled, M, w->K)) return MQ_ERR_CUDA;
+    mq::GemmArgs a;
+    a.s_enc_a = a_s_enc_dev;
+    a.s_enc_b = w->s_enc;
+    a.y = y_bf16;
+    a.ldy = ldy;
+    a.M = static_cast<int>(M);
+    a.N = static_cast<int>(w->N);
+    a.K = static_cast<int>(w->K);
+    a.amax_partials = nullptr;
+    a.err = d->err;
+    a.wait_ns = static_cast<unsigned long long>(wait_limit_us) * 1000ull;
+    a.withhold_release = 1;
+    return cuda_status(mq::launch_gemm_nvf4(ta, w->tmap, tsa, w->tmap_sf, a, false, d->num_sms, nullptr,
+                                            stream));
 }
 
 mq_status mq_gemm_nvfp4_swiglu(const uint8_t *a_codes, const uint8_t *a_sf_swizzled,

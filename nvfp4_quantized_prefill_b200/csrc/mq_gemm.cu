@@ -99,6 +99,8 @@ struct Params {
     float *amax_partials;
     unsigned *err;
     int tma_store;        // 1: outputs leave through TMA stores via shared memory
+    unsigned long long wait_ns;   // bound of every wait (kWaitLimitNs outside tests)
+    int withhold_release;         // test only: the first stage is never released
 };
 
 __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int &tm, int &tn) {
@@ -113,10 +115,11 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int
 
 // Waits (time-bounded, ignoring the abort flag) so that in-flight asynchronous
 // work signalling `bar` has landed before the CTA exits.
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, unsigned *err) {
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, unsigned *err,
+                                           unsigned long long limit_ns) {
     unsigned long long t0 = global_timer_ns();
     while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (global_timer_ns() - t0 > limit_ns) {
             atomicOr(err, kDevErrTimeout);
             return;
         }
@@ -245,7 +248,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int a_row = tm * 256 + static_cast<int>(rank) * 128;
             const int a_sf = (2 * tm + static_cast<int>(rank)) * p.sf_ktiles;
             for (int kt = 0; kt < p.k_tiles; ++kt) {
-                if (!warp_mbar_wait(empty0 + 8u * stage, phase ^ 1u, abort_flag, p.err)) {
+                if (!warp_mbar_wait(empty0 + 8u * stage, phase ^ 1u, abort_flag, p.err, p.wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -280,8 +283,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // both CTAs' loads of every armed stage land before the pair may exit
         for (int s2 = 0; s2 < kStages; ++s2)
             if (armed & (1u << s2)) {
-                drain_wait(sfd_full0 + 8u * s2, (armed_parity >> s2) & 1u, p.err);
-                drain_wait(bar0 + 8u * s2, (armed_parity >> s2) & 1u, p.err);
+                drain_wait(sfd_full0 + 8u * s2, (armed_parity >> s2) & 1u, p.err, p.wait_ns);
+                drain_wait(bar0 + 8u * s2, (armed_parity >> s2) & 1u, p.err, p.wait_ns);
             }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -291,13 +294,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
             for (int t = pair; t < num_tiles && ok; t += npairs) {
-                if (!warp_mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag, p.err)) break;
+                if (!warp_mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag, p.err, p.wait_ns)) break;
                 tc_fence_after();
                 for (int kt = 0; kt < p.k_tiles; ++kt) {
                     // the stage's scales are in TMEM and both CTAs' operands
                     // landed: the copiers commit sf_full only after seeing the
                     // operand barrier, so this is the one wait per stage
-                    if (!warp_mbar_wait(sf_full0 + 8u * stage, phase, abort_flag, p.err)) {
+                    if (!warp_mbar_wait(sf_full0 + 8u * stage, phase, abort_flag, p.err, p.wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -307,7 +310,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const uint32_t sB = sA + kABytes;
                     const uint32_t tsfa = tmem + kSfCol + stage * kSfColsPerStage;
                     const uint32_t tsfb = tsfa + 16u;
-                    if (natoms == 4) {
+                    if (p.withhold_release && t == pair && kt == 0) {
+                        // test only: the stage's MMAs without the commit that
+                        // frees it, so the producer's next wait on it runs out
+                        for (int kb = 0; kb < natoms; ++kb)
+                            warp_mma_nvf4_pair(tmem, sdesc_kmajor_sw128(sA + 32u * kb),
+                                               sdesc_kmajor_sw128(sB + 32u * kb), idesc, tsfa + 4u * kb,
+                                               tsfb + 8u * kb, kb != 0 ? 1u : 0u);
+                    } else if (natoms == 4) {
                         warp_mma4_commit_pair(tmem, sdesc_kmajor_sw128(sA), sdesc_kmajor_sw128(sB), idesc,
                                               tsfa, tsfb, kt != 0 ? 1u : 0u, empty0 + 8u * stage,
                                               kPairMask);
@@ -330,7 +340,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
             // every MMA issued by this warp completes before TMEM is freed
             warp_commit_pair(drain_bar);
-            drain_wait(drain_bar, 0, p.err);
+            drain_wait(drain_bar, 0, p.err, p.wait_ns);
         }
     } else {
         // ------------------------------------------------------------ scale copiers
@@ -344,7 +354,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             bool ok = true;
             for (int t = pair; t < num_tiles && ok; t += npairs) {
                 for (int kt = 0; kt < p.k_tiles; ++kt) {
-                    if (!warp_mbar_wait(sfd_full0 + 8u * stage, phase, abort_flag, p.err)) {
+                    if (!warp_mbar_wait(sfd_full0 + 8u * stage, phase, abort_flag, p.err, p.wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -369,7 +379,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                     // the operands too have landed when sf_full completes, so
                     // the MMA thread waits on one barrier per stage
-                    if (!warp_mbar_wait(bar0 + 8u * stage, phase, abort_flag, p.err)) {
+                    if (!warp_mbar_wait(bar0 + 8u * stage, phase, abort_flag, p.err, p.wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -381,7 +391,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
             }
             warp_commit_pair(sf_drain_bar);
-            drain_wait(sf_drain_bar, 0, p.err);
+            drain_wait(sf_drain_bar, 0, p.err, p.wait_ns);
         }
     }
     } else {
@@ -446,7 +456,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int tm, tn;
             tile_coords(t, p.tiles_m, p.tiles_n, tm, tn);
             // warp-uniform decision: the TMEM loads below are .sync.aligned
-            const bool got = __all_sync(0xFFFFFFFFu, mbar_wait(acc_full, acc_phase, abort_flag, p.err));
+            const bool got = __all_sync(0xFFFFFFFFu, mbar_wait(acc_full, acc_phase, abort_flag, p.err, p.wait_ns));
             if (got) tc_fence_after();
             const int row0 = tm * 256 + static_cast<int>(rank) * 128 + sub * 32;
             const int row = row0 + lane;
@@ -649,6 +659,8 @@ cudaError_t launch_gemm_nvf4(const CUtensorMap &tmap_a, const CUtensorMap &tmap_
     p.k_tiles = (p.sf_ktiles + 3) / 4;
     p.amax_partials = a.amax_partials;
     p.err = a.err;
+    p.wait_ns = a.wait_ns ? a.wait_ns : kWaitLimitNs;
+    p.withhold_release = a.withhold_release;
     const int tiles = p.tiles_m * p.tiles_n;
     const int max_pairs = num_sms / 2;
     int pairs = tiles < max_pairs ? tiles : max_pairs;

@@ -82,6 +82,8 @@ struct GemmArgs {
     int M, N, K;              // N = weight rows (gate+up rows with SwiGLU)
     float *amax_partials;     // SwiGLU: one max |h| per CTA
     unsigned *err;            // device error word
+    unsigned long long wait_ns = 0;   // 0: the standard bound of every wait
+    int withhold_release = 0;         // test only (mq_debug.h): never free the first stage
 };
 
 // Launches the tcgen05 GEMM; *grid_out receives the CTA count (the number of

@@ -59,14 +59,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Returns false (after latching kDevErrTimeout and raising *abort) if it takes
 // longer than kWaitLimitNs, or if another role already raised *abort.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
-                                          unsigned *err) {
+                                          unsigned *err, unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     unsigned long long t0 = global_timer_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 255u) == 0) {
             if (*abort) return false;
-            if (global_timer_ns() - t0 > kWaitLimitNs) {
+            if (global_timer_ns() - t0 > limit_ns) {
                 atomicOr(err, kDevErrTimeout);
                 *abort = 1;
                 return false;
@@ -366,8 +366,9 @@ __device__ __forceinline__ void warp_commit_pair(uint32_t bar) {
 
 // Warp-uniform bounded wait: every lane polls; the warp agrees on the result.
 __device__ __forceinline__ bool warp_mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
-                                               unsigned *err) {
-    return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort, err));
+                                               unsigned *err,
+                                               unsigned long long limit_ns = kWaitLimitNs) {
+    return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort, err, limit_ns));
 }
 
 // ---- tcgen05 -------------------------------------------------------------------

@@ -31,10 +31,28 @@ def test_header_declares_expected_entry_points():
         assert n in names
 
 
+def debug_header_functions():
+    src = open(os.path.join(ROOT, "include", "mq_debug.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return set(re.findall(r"\b(mq_[a-z0-9_]+)\s*\(", src))
+
+
 def test_library_exports_every_header_symbol(lib):
-    for name in header_functions():
+    for name in header_functions() | debug_header_functions():
         assert hasattr(lib, name), name
         assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_debug_entry_point_checks_its_arguments_on_the_host(lib):
+    f = lib.mq_debug_gemm_withhold_release
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                                          ctypes.c_int64, ctypes.c_uint32, ctypes.c_void_p]
+    assert debug_header_functions() == {"mq_debug_gemm_withhold_release"}
+    assert not (debug_header_functions() & header_functions())   # not in the public header
+    assert f(None, 16, 16, 8, 16, 16, 8, 20000, None) == 1       # null pointer
+    assert f(16, 16, 16, 8, 16, 16, 8, 999, None) == 1           # wait limit below 1 ms
+    assert f(16, 16, 16, 8, None, 16, 8, 20000, None) == 1       # no weight handle
 
 
 def test_binding_covers_header(lib):
