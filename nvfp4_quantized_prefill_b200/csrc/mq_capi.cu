@@ -672,6 +672,12 @@ mq_status mq_decode_linear_nvfp4(const mq_weight *w, const void *x_bf16, int64_t
     DeviceInfo *d = nullptr;
     st = device_info(&d);
     if (st != MQ_OK) return st;
+    // 1 to 4 tokens on a weight of up to 2^25 elements: the CUDA-core stream
+    // (the tensor-core kernel's fixed per-CTA path costs more there); larger
+    // weights stream faster through the tensor-core kernel below
+    if (mq::decode_nvf4_gemv_fits(M, w->K) && w->N * w->K <= (int64_t(1) << 25))
+        return cuda_status(mq::launch_decode_nvf4_gemv(w->codes, w->sf, w->s_enc, w->N, w->K, x_bf16,
+                                                       M, y_bf16, d->num_sms, stream));
     const size_t tok_bytes = static_cast<size_t>(M) * static_cast<size_t>(w->K) * 9u / 16u;
     const bool tc_fits = M <= mq::kDecodeTcTokens && tok_bytes + 15u <= mq::kDecodeTcTokenSmem;
     // the tensor-core kernel (quantizes the tokens itself, one pass over the

@@ -148,6 +148,15 @@ cudaError_t launch_decode_nvf4(const uint8_t *x_codes, const uint8_t *x_sf, cons
                                const uint8_t *w_sf, const float *s_enc_w, int64_t N, int64_t K,
                                void *y, void *scratch, int num_sms, cudaStream_t s);
 
+// W4A4 decode on the CUDA cores for 1 to 4 tokens (mq_decode_gemv4.cu): a
+// stream over the weight's NVFP4 bytes with the tokens quantized in shared
+// memory (M x ceil(K / 1024) x 2 KB of it, at most kDecodeGemvTokenSmem).
+constexpr int64_t kDecodeGemvTokenSmem = 96 * 1024;
+bool decode_nvf4_gemv_fits(int64_t M, int64_t K);
+cudaError_t launch_decode_nvf4_gemv(const uint8_t *w_codes, const uint8_t *w_sf, const float *s_enc_w,
+                                    int64_t N, int64_t K, const void *x_bf16, int64_t M, void *y,
+                                    int num_sms, cudaStream_t s);
+
 // W4A4 decode on the tcgen05 tensor cores (mq_decode_tc.cu) for up to
 // kDecodeTcTokens BF16 tokens x [M, K] whose NVFP4 form (M K 9 / 16 bytes)
 // fits in kDecodeTcTokenSmem; the kernel quantizes them itself.  tmap_w is
