@@ -15,9 +15,13 @@ kernel to write back.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference ...   (the CPU oracle, bounded sample)
+  python bench.py --sharded ...          (the batch split by tokens across ranks)
+  python bench.py --profile-case NAME    (one small case for an ncu capture)
 
 Multi-GPU: one process per GPU (torchrun), independent replicas (the layer
-needs no exchange); value = work of all ranks / max-over-ranks time.
+needs no exchange); value = work of all ranks / max-over-ranks time.  With
+--sharded the batch is split by tokens and the ranks all-reduce one float per
+activation (the tensor scale); value = the batch's work / max-over-ranks time.
 """
 from __future__ import annotations
 
@@ -164,6 +168,14 @@ def reduce_over_ranks(v: float, world: int, op: str) -> float:
     t = torch.tensor([v], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=getattr(torch.distributed.ReduceOp, op))
     return float(t.item())
+
+
+def aggregate_sharded(batch_flops: float, ms_local: float, world: int):
+    """Whole-job throughput of a batch split by tokens across the ranks: the
+    batch's work (counted once) over the slowest rank's time (strong
+    scaling).  Returns (tflops, max_ms)."""
+    max_ms = reduce_over_ranks(ms_local, world, "MAX")
+    return batch_flops / (max_ms * 1e-3) / 1e12, max_ms
 
 
 def aggregate(flops_local: float, prefill_ms_local: float, world: int):
@@ -1029,6 +1041,135 @@ def run_gpu(args, wl, world, rank):
     return out, P
 
 
+def run_sharded(args, wl, world, rank):
+    """The workload's prefill with the batch split by tokens across the ranks
+    (row blocks of every activation; weights replicated): per activation and
+    rank, shard amax -> one float all-reduced (max) over NCCL -> quantize with
+    the batch's tensor scale -> GEMM, so every rank's rows are the single-GPU
+    result.  Timed like the replica leg: CUDA events at the step boundaries,
+    L2 flushed between steps, max over ranks; value = the batch's FLOPs over
+    the slowest rank's time."""
+    from nvfp4_quantized_prefill_b200 import binding as mq
+    from nvfp4_quantized_prefill_b200 import sharded
+    mq.lib()
+    if wl.swiglu or wl.chunks > 1 or wl.rmsnorm:
+        raise SystemExit("--sharded runs plain projection workloads (e.g. llama3_8b_qkv_o)")
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    M = wl.M
+    lo, hi = M * rank // world, M * (rank + 1) // world
+    Ml = hi - lo
+    ws_full = workloads.layer_weights(wl, device=str(dev))
+    W = [mq.Weight(w) for w in ws_full]
+    # every rank draws the same batch (same seed) and keeps its rows
+    xs = [workloads.layer_activation(wl, w.shape[1], i, device=str(dev))[lo:hi].contiguous()
+          for i, w in enumerate(ws_full)]
+    ys = [torch.empty(Ml, Wi.N, dtype=torch.bfloat16, device=dev) for Wi in W]
+    shard_ws = [sharded.ShardWorkspace.create(Ml, Wi.K, device=dev) for Wi in W]
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(256 << 20, dtype=torch.uint8, device=dev)
+    sink = torch.empty((), dtype=torch.int64, device=dev)
+
+    def step():
+        for Wi, x, y, sw in zip(W, xs, ys, shard_ws):
+            sharded.shard_amax(x, sw, stream)
+            if world > 1:
+                sharded.exchange_amax(sw.amax)
+            sharded.shard_finish(Wi, x, y, sw, stream)
+
+    for _ in range(args.warmup):
+        flush_w.zero_()
+        torch.sum(flush_r, dim=0, dtype=torch.int64, out=sink)
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    barrier(world)
+    torch.cuda.synchronize()
+    with clocks:
+        time.sleep(0.3)
+        for a, b in evs:
+            flush_w.zero_()
+            torch.sum(flush_r, dim=0, dtype=torch.int64, out=sink)
+            a.record(stream)
+            step()
+            b.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    if mq.mq_check(stream) != 0:
+        raise RuntimeError("device error during the sharded steps")
+    ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    batch_flops = sum(2.0 * M * w.shape[0] * w.shape[1] for w in ws_full)
+    value, max_ms = aggregate_sharded(batch_flops, ms, world)
+    pk = peaks()
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(max_ms, 4),
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 codes, e4m3 per-16 scales, fp32 tensor scale) -> fp32 acc -> bf16",
+        "data": "synthetic (seeded recipe, random-init weights of the named shapes)",
+        "config": {"workload": wl.name, "workload_key": args.workload, "tokens": M,
+                   "tokens_per_rank": Ml,
+                   "linears": [{"name": l.name, "N": l.N, "K": l.K} for l in wl.linears],
+                   "parallelism": f"token-sharded x{world}: rows split across ranks, weights "
+                                  "replicated, one float all-reduced (max) per activation",
+                   "l2": "flushed between steps (outside the timed intervals)"},
+        "fp4_peak_frac": round(value / (world * pk["bf16"] * FP4_OVER_BF16), 4),
+        "e2e": None,
+        "e2e_note": "the sharded leg times the device path only; e2e is reported by the "
+                    "default (replica) leg",
+        "gpu_launches": args.steps * len(W) * 4,
+        "clocks": clocks.summary(),
+    }
+    for Wi in W:
+        Wi.free()
+    return out
+
+
+def profile_case(name: str):
+    """Runs one small case a few times for a kernel capture (ncu -k ... -c 1):
+    attention_prefill (4096 tokens, 8 query / 2 KV heads, head dim 128),
+    attention_decode (1 token over that cache), decode_nvfp4 (one token
+    through the Llama-3-8B QKV weight, W4A4)."""
+    from nvfp4_quantized_prefill_b200 import binding as mq
+    mq.lib()
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(9)
+    if name.startswith("attention"):
+        M, H, Hkv, D = 4096, 8, 2, 128
+        qkv = torch.randn(M + 1, (H + 2 * Hkv) * D, device=dev, generator=g).to(torch.bfloat16)
+        kc = torch.zeros(Hkv, M + 8, D, dtype=torch.bfloat16, device=dev)
+        vc = torch.zeros_like(kc)
+        o = torch.empty(M, H * D, dtype=torch.bfloat16, device=dev)
+        part = torch.empty(mq.MQ_AMAX_PARTIALS_MAX, dtype=torch.float32, device=dev)
+        for _ in range(3):
+            mq.mq_attention_prefill_bf16(qkv[:M], M, H, Hkv, D, kc, vc, M + 8, o, part)
+        if name == "attention_decode":
+            ot = torch.empty(1, H * D, dtype=torch.bfloat16, device=dev)
+            nb = mq.mq_attention_decode_workspace_bytes(1, M, H, Hkv, D)
+            ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+            for _ in range(3):
+                mq.mq_attention_decode_bf16(qkv[M:M + 1], 1, M, H, Hkv, D, kc, vc, M + 8, ot, ws, nb)
+    elif name == "decode_nvfp4":
+        w = (torch.randn(6144, 4096, device=dev, generator=g) * 0.02).to(torch.bfloat16)
+        W = mq.Weight(w)
+        x = torch.randn(1, 4096, device=dev, generator=g).to(torch.bfloat16)
+        y = torch.empty(1, 6144, dtype=torch.bfloat16, device=dev)
+        nb = mq.mq_workspace_bytes(1, 4096)
+        ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            mq.mq_decode_linear_nvfp4(W.handle, x, 1, y, ws, nb)
+    else:
+        raise SystemExit(f"unknown profile case {name}")
+    torch.cuda.synchronize()
+    if mq.mq_check() != 0:
+        raise RuntimeError("device error in the profile case")
+    print(json.dumps({"profile_case": name, "ok": True}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -1043,8 +1184,17 @@ def main():
                     help="skip the lighter measurement of the other workloads")
     ap.add_argument("--config-steps", type=int, default=5,
                     help="timed steps per workload in per_config")
+    ap.add_argument("--profile-case", default=None,
+                    choices=["attention_prefill", "attention_decode", "decode_nvfp4"],
+                    help="run one small case for a kernel capture and exit")
+    ap.add_argument("--sharded", action="store_true",
+                    help="split the batch by tokens across the ranks (one float all-reduced "
+                         "per activation) instead of running replicas")
     args = ap.parse_args()
     wl = workloads.WORKLOADS[args.workload]
+    if args.profile_case:
+        profile_case(args.profile_case)
+        return
 
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
@@ -1076,6 +1226,13 @@ def main():
         return
 
     world, rank, local = dist_setup()
+    if args.sharded:
+        out = run_sharded(args, wl, world, rank)
+        if rank == 0:
+            print(json.dumps(out))
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
     out, P = run_gpu(args, wl, world, rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not wl.swiglu and wl.chunks == 1 and not wl.rmsnorm:
         import oracle
