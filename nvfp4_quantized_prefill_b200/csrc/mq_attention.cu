@@ -393,10 +393,15 @@ EncodeFn encode_fn() {
 // FP32 throughout (scores, weights, accumulation); BF16 output.
 
 constexpr int kDecChunk = 128;            // keys per sub-chunk in shared memory
-// 128-key sub-chunks per CTA: four (512 keys) for up to 8 query rows, where a
-// CTA's work is mostly the cache read; one for more rows, where the FP32
-// arithmetic per key grows and more CTAs share it
-__host__ __device__ constexpr int dec_sub(int64_t rows) { return rows <= 8 ? 4 : 1; }
+// 128-key sub-chunks per CTA: at most four (512 keys) for up to 8 query rows,
+// where a CTA's work is mostly the cache read; one for more rows, where the
+// FP32 arithmetic per key grows and more CTAs share it.  Fewer when the cache
+// is short: the span shrinks until the CTAs (spans x KV heads) cover the SMs.
+int dec_sub(int64_t rows, int64_t n_keys, int64_t Hkv, int num_sms) {
+    for (int n_sub = rows <= 8 ? 4 : 1; n_sub > 1; n_sub /= 2)
+        if ((n_keys + kDecChunk * n_sub - 1) / (kDecChunk * n_sub) * Hkv >= num_sms) return n_sub;
+    return 1;
+}
 constexpr int kDecThreads = 256;
 constexpr int kDecMaxRows = 64;           // query rows per KV head (group size x tokens)
 constexpr int kKPad = kD + 2;             // padded K row in shared memory (conflict-free dot products)
@@ -601,9 +606,9 @@ __global__ void __launch_bounds__(kD) attention_combine_kernel(const DecodeParam
 }  // namespace
 
 size_t attention_decode_workspace_bytes(int64_t m, int64_t pos0, int64_t H, int64_t Hkv) {
+    // sized for one-sub-chunk spans, the most a launch uses on any GPU
     const int64_t rows = H / Hkv * m;
-    const int64_t span = kDecChunk * dec_sub(rows);
-    const int64_t n_chunks = (pos0 + m + span - 1) / span;
+    const int64_t n_chunks = (pos0 + m + kDecChunk - 1) / kDecChunk;
     return static_cast<size_t>(Hkv * n_chunks * rows * (2 + kD)) * sizeof(float);
 }
 
@@ -611,7 +616,7 @@ int attention_decode_max_rows() { return kDecMaxRows; }
 
 cudaError_t launch_attention_decode(const void *qkv, int64_t m, int64_t pos0, int64_t H, int64_t Hkv,
                                     void *k_cache, void *v_cache, int64_t S_max, void *o, void *ws,
-                                    cudaStream_t s) {
+                                    int num_sms, cudaStream_t s) {
     DecodeParams p;
     p.qkv = static_cast<const __nv_bfloat16 *>(qkv);
     p.k_cache = static_cast<__nv_bfloat16 *>(k_cache);
@@ -624,7 +629,7 @@ cudaError_t launch_attention_decode(const void *qkv, int64_t m, int64_t pos0, in
     p.Hkv = static_cast<int>(Hkv);
     p.S_max = static_cast<int>(S_max);
     p.rows = static_cast<int>(H / Hkv * m);
-    p.n_sub = dec_sub(p.rows);
+    p.n_sub = dec_sub(p.rows, pos0 + m, Hkv, num_sms);
     p.n_chunks = static_cast<int>((pos0 + m + kDecChunk * p.n_sub - 1) / (kDecChunk * p.n_sub));
     cudaError_t e = launch_pdl(kv_append_kernel, dim3(p.m, p.Hkv), dim3(32), 0, s, p);
     if (e != cudaSuccess) return e;
