@@ -387,29 +387,31 @@ EncodeFn encode_fn() {
 // Decode step: m new tokens at positions pos0 .. pos0 + m - 1.  Their K / V
 // rows are appended to the cache, then each query attends over keys
 // 0 .. pos0 + t of the cache.  Memory-bound (the cache is read once): the
-// keys are split into 128-key chunks across CTAs (one CTA per chunk and KV
-// head, all of the group's query rows at once), each CTA leaves (max, sum,
-// unnormalised o) per query row, and a combine pass merges the chunks.
-// FP32 throughout (scores, weights, accumulation); BF16 output.
+// keys are split into spans of 64-key blocks across many small CTAs (one CTA
+// per span and KV head, all of the group's query rows at once, so each K / V
+// byte crosses HBM once per step), each CTA leaves (max, sum, unnormalised o)
+// per query row, and a combine pass merges the spans.  FP32 throughout
+// (scores, weights, accumulation); BF16 output.
 
-constexpr int kDecChunk = 128;            // keys per sub-chunk in shared memory
-// 128-key sub-chunks per CTA: at most four (512 keys) for up to 8 query rows,
-// where a CTA's work is mostly the cache read; one for more rows, where the
-// FP32 arithmetic per key grows and more CTAs share it.  Fewer when the cache
-// is short: the span shrinks until the CTAs (spans x KV heads) cover the SMs.
-int dec_sub(int64_t rows, int64_t n_keys, int64_t Hkv, int num_sms) {
-    for (int n_sub = rows <= 8 ? 4 : 1; n_sub > 1; n_sub /= 2)
-        if ((n_keys + kDecChunk * n_sub - 1) / (kDecChunk * n_sub) * Hkv >= num_sms) return n_sub;
-    return 1;
-}
-constexpr int kDecThreads = 256;
+constexpr int kDecKeys = 64;              // keys per block
+constexpr int kDecThreads = 128;          // 4 warps: 16 keys each for the scores, one dimension each for P.V
 constexpr int kDecMaxRows = 64;           // query rows per KV head (group size x tokens)
-constexpr int kKPad = kD + 2;             // padded K row in shared memory (conflict-free dot products)
-// shared memory: the chunk's K (padded rows) and V, then per query row its
-// FP32 query and its chunk of scores / weights (sized by the row count, so
-// that a one-token step fits three CTAs on an SM)
-constexpr uint32_t kDecSmemFixed = kDecChunk * kKPad * 2 + kDecChunk * kD * 2;
-constexpr uint32_t kDecSmemPerRow = kD * 4 + kDecChunk * 4;
+#ifndef MQ_DEC_MAX_CTAS
+#define MQ_DEC_MAX_CTAS 2048
+#endif
+constexpr int kDecMaxCtas = MQ_DEC_MAX_CTAS;  // spans x KV heads stay below this (bounds the workspace)
+// shared memory: the block's V, then per query row its FP32 query and its
+// block of scores / weights (sized by the row count)
+constexpr uint32_t kDecSmemFixed = kDecKeys * kD * 2;
+constexpr uint32_t kDecSmemPerRow = kD * 4 + kDecKeys * 4;
+
+// 64-key blocks per span: one, unless the cache is long enough that the
+// spans x KV heads would pass kDecMaxCtas
+__host__ __device__ constexpr int64_t dec_span_blocks(int64_t n_keys, int64_t Hkv) {
+    const int64_t blocks = (n_keys + kDecKeys - 1) / kDecKeys;
+    const int64_t sb = (blocks * Hkv + kDecMaxCtas - 1) / kDecMaxCtas;
+    return sb < 1 ? 1 : sb;
+}
 
 struct DecodeParams {
     const __nv_bfloat16 *qkv;   // [m, (H + 2 Hkv) * 128]
@@ -418,7 +420,7 @@ struct DecodeParams {
     __nv_bfloat16 *o;           // [m, H * 128]
     float *part;                // [Hkv, n_chunks, rows, 2 + 128]
     int m, pos0, H, Hkv, S_max, n_chunks, rows;
-    int n_sub;                  // 128-key sub-chunks per CTA
+    int span_blocks;            // 64-key blocks per CTA
 };
 
 // Copies the new tokens' K and V rows into the cache (grid m x Hkv, 32 threads).
@@ -438,21 +440,41 @@ __global__ void __launch_bounds__(32) kv_append_kernel(const DecodeParams p) {
         reinterpret_cast<uint4 *>(p.v_cache + dst)[lane - 16] = src_v[lane - 16];
 }
 
+__device__ __forceinline__ uint4 ldg_nc_v4(const void *ptr) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(ptr));
+    return v;
+}
+
+// 16 bytes global -> shared, asynchronously; src_bytes = 0 fills zeros
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 // kRows: the largest query-row count this instance serves (its share of o in
 // registers scales with it)
 template <int kRows>
-__global__ void __launch_bounds__(kDecThreads, 2) attention_decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kDecThreads) attention_decode_kernel(const DecodeParams p) {
     extern __shared__ __align__(16) uint8_t dsm[];
-    __nv_bfloat16 *ks = reinterpret_cast<__nv_bfloat16 *>(dsm);                       // [128][130]
-    __nv_bfloat16 *vs = ks + kDecChunk * kKPad;                                          // [128][128]
-    float *qs = reinterpret_cast<float *>(vs + kDecChunk * kD);                          // [rows][128]
-    float *ss = qs + p.rows * kD;                                                        // [rows][128]
+    __nv_bfloat16 *vs = reinterpret_cast<__nv_bfloat16 *>(dsm);                        // [64][128]
+    float *qs = reinterpret_cast<float *>(dsm + kDecSmemFixed);                          // [rows][128]
+    float *ps = qs + p.rows * kD;                                                        // [rows][64]
     __shared__ float m_run[kDecMaxRows], l_run[kDecMaxRows], alpha[kDecMaxRows];
     const int c = blockIdx.x, g = blockIdx.y, tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int group = p.H / p.Hkv;
     const int n_keys = p.pos0 + p.m;
     const int cols = (p.H + 2 * p.Hkv) * kD;
+    const __nv_bfloat16 *kbase = p.k_cache + static_cast<int64_t>(g) * p.S_max * kD;
+    const __nv_bfloat16 *vbase = p.v_cache + static_cast<int64_t>(g) * p.S_max * kD;
+    const uint32_t vs_addr = smem_u32(vs);
     griddep_wait();            // the appended rows and the queries are in place
     griddep_launch_dependents();
     // the group's query rows: row rr = hh * m + t (head g * group + hh, token t)
@@ -464,97 +486,91 @@ __global__ void __launch_bounds__(kDecThreads, 2) attention_decode_kernel(const 
         m_run[rr] = -INFINITY;
         l_run[rr] = 0.0f;
     }
-    // this thread's share of o: dimension d of rows half, half + 2, ...
-    const int d = tid & (kD - 1), half = tid >> 7;
-    float acc[kRows / 2];
+    // scores: this lane takes key kk of the block, dimensions [64 kh, 64 kh + 64)
+    const int kk = warp * 16 + (lane & 15), kh = lane >> 4;
+    // P.V: this thread's dimension of every row
+    const int d = tid;
+    float acc[kRows];
 #pragma unroll
-    for (int i = 0; i < kRows / 2; ++i) acc[i] = 0.0f;
-    // the CTA's keys: n_sub 128-key sub-chunks, merged on the fly
-    for (int sc = 0; sc < p.n_sub; ++sc) {
-        const int key0 = (c * p.n_sub + sc) * kDecChunk;
-        const int nk = min(kDecChunk, n_keys - key0);
-        if (nk <= 0) break;    // uniform over the CTA
-        __syncthreads();       // the previous sub-chunk's K, V and weights are consumed
-        for (int i = tid; i < kDecChunk * (kD / 8); i += kDecThreads) {
-            const int k = i / (kD / 8), d8 = (i % (kD / 8)) * 8;
-            uint4 kv = make_uint4(0, 0, 0, 0), vv = kv;
-            if (k < nk) {
-                const int64_t off = (static_cast<int64_t>(g) * p.S_max + key0 + k) * kD + d8;
-                kv = *reinterpret_cast<const uint4 *>(p.k_cache + off);
-                vv = *reinterpret_cast<const uint4 *>(p.v_cache + off);
-            }
-            const uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e)   // the padded K rows are only 4-byte aligned
-                *reinterpret_cast<uint32_t *>(ks + k * kKPad + d8 + 2 * e) = w[e];
-            *reinterpret_cast<uint4 *>(vs + k * kD + d8) = vv;
-        }
-        __syncthreads();
-        // scores: thread -> one key, every other row
+    for (int i = 0; i < kRows; ++i) acc[i] = 0.0f;
+    for (int b = 0; b < p.span_blocks; ++b) {
+        const int key0 = (c * p.span_blocks + b) * kDecKeys;
+        if (key0 >= n_keys) break;   // uniform over the CTA
+        const int nk = min(kDecKeys, n_keys - key0);
+        __syncthreads();             // the previous block's V and weights are consumed
+        // this lane's half key row into registers (zeros past the cache's end)
+        uint32_t kr[32];
         {
-            const int k = tid & (kDecChunk - 1);
-            uint32_t kr[kD / 2];   // the key's 128 values, two BF16 a register
+            const int key = kk < nk ? key0 + kk : key0;
+            const uint4 *src = reinterpret_cast<const uint4 *>(kbase + static_cast<int64_t>(key) * kD + kh * 64);
 #pragma unroll
-            for (int dd = 0; dd < kD; dd += 2) kr[dd / 2] = *reinterpret_cast<const uint32_t *>(ks + k * kKPad + dd);
-            const int pos = key0 + k;
-            for (int rr = half; rr < p.rows; rr += 2) {
-                const float *q = qs + rr * kD;
-                float a0 = 0.0f, a1 = 0.0f;
-#pragma unroll
-                for (int dd = 0; dd < kD; dd += 4) {
-                    const float4 qv = *reinterpret_cast<const float4 *>(q + dd);
-                    a0 = fmaf(qv.x, __uint_as_float(kr[dd / 2] << 16), a0);
-                    a1 = fmaf(qv.y, __uint_as_float(kr[dd / 2] & 0xFFFF0000u), a1);
-                    a0 = fmaf(qv.z, __uint_as_float(kr[dd / 2 + 1] << 16), a0);
-                    a1 = fmaf(qv.w, __uint_as_float(kr[dd / 2 + 1] & 0xFFFF0000u), a1);
-                }
-                const int t = rr % p.m;
-                ss[rr * kDecChunk + k] = (k < nk && pos <= p.pos0 + t) ? (a0 + a1) * kScaleLog2 : -INFINITY;
+            for (int j = 0; j < 8; ++j) {
+                uint4 v = ldg_nc_v4(src + j);
+                if (kk >= nk) v = make_uint4(0, 0, 0, 0);
+                kr[4 * j] = v.x; kr[4 * j + 1] = v.y; kr[4 * j + 2] = v.z; kr[4 * j + 3] = v.w;
             }
+        }
+        // the block's V into shared memory, asynchronously (zeros past the end)
+        for (int i = tid; i < kDecKeys * (kD / 8); i += kDecThreads) {
+            const int k = i >> 4, c16 = i & 15;
+            const int key = k < nk ? key0 + k : key0;
+            cp_async16(vs_addr + static_cast<uint32_t>(i) * 16u, vbase + static_cast<int64_t>(key) * kD + c16 * 8,
+                       k < nk ? 16u : 0u);
+        }
+        // scores in the base-2 exponent domain; masked: past the cache or
+        // after the row's own position
+        const int pos = key0 + kk;
+        for (int r = 0; r < p.rows; ++r) {
+            const float *q = qs + r * kD + kh * 64;
+            float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+                const float4 qv = *reinterpret_cast<const float4 *>(q + 2 * j);
+                a0 = fmaf(qv.x, __uint_as_float(kr[j] << 16), a0);
+                a1 = fmaf(qv.y, __uint_as_float(kr[j] & 0xFFFF0000u), a1);
+                a0 = fmaf(qv.z, __uint_as_float(kr[j + 1] << 16), a0);
+                a1 = fmaf(qv.w, __uint_as_float(kr[j + 1] & 0xFFFF0000u), a1);
+            }
+            float sc = a0 + a1;
+            sc += __shfl_xor_sync(0xFFFFFFFFu, sc, 16);
+            const int t = r % p.m;
+            if (lane < 16) ps[r * kDecKeys + kk] = (kk < nk && pos <= p.pos0 + t) ? sc * kScaleLog2 : -INFINITY;
         }
         __syncthreads();
         // per row: running maximum, weights 2^(x - max), running sum (a warp a row)
-        for (int rr = warp; rr < p.rows; rr += kDecThreads / 32) {
-            float x[4], mx = -INFINITY;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                x[e] = ss[rr * kDecChunk + lane + 32 * e];
-                mx = fmaxf(mx, x[e]);
-            }
+        for (int r = warp; r < p.rows; r += kDecThreads / 32) {
+            const float x0 = ps[r * kDecKeys + lane], x1 = ps[r * kDecKeys + lane + 32];
+            float mx = fmaxf(x0, x1);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-            const float m_old = m_run[rr];
+            const float m_old = m_run[r];
             const float m_new = fmaxf(m_old, mx);
-            float sum = 0.0f;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float w = m_new == -INFINITY ? 0.0f : exp2f(x[e] - m_new);
-                ss[rr * kDecChunk + lane + 32 * e] = w;
-                sum += w;
-            }
+            const float w0 = m_new == -INFINITY ? 0.0f : exp2f(x0 - m_new);
+            const float w1 = m_new == -INFINITY ? 0.0f : exp2f(x1 - m_new);
+            ps[r * kDecKeys + lane] = w0;
+            ps[r * kDecKeys + lane + 32] = w1;
+            float sum = w0 + w1;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
-            __syncwarp();
             if (lane == 0) {
                 const float a = (m_old == -INFINITY) ? 0.0f : exp2f(m_old - m_new);
-                alpha[rr] = a;
-                l_run[rr] = l_run[rr] * a + sum;
-                m_run[rr] = m_new;
+                alpha[r] = a;
+                l_run[r] = l_run[r] * a + sum;
+                m_run[r] = m_new;
             }
         }
+        cp_async_wait_all();
         __syncthreads();
-        // o: rescale, then add this sub-chunk's weighted values -- each value
-        // loaded once for all of this thread's rows (weights are broadcast)
+        // o: rescale, then add the block's weighted values (each value read
+        // once for all rows; the weights are broadcast)
 #pragma unroll
-        for (int i = 0; i < kRows / 2; ++i)
-            if (half + 2 * i < p.rows) acc[i] *= alpha[half + 2 * i];
+        for (int i = 0; i < kRows; ++i)
+            if (i < p.rows) acc[i] *= alpha[i];
         for (int k = 0; k < nk; ++k) {
             const float v = __bfloat162float(vs[k * kD + d]);
 #pragma unroll
-            for (int i = 0; i < kRows / 2; ++i) {
-                const int rr = half + 2 * i;
-                if (rr < p.rows) acc[i] = fmaf(ss[rr * kDecChunk + k], v, acc[i]);
-            }
+            for (int i = 0; i < kRows; ++i)
+                if (i < p.rows) acc[i] = fmaf(ps[i * kDecKeys + k], v, acc[i]);
         }
     }
     __syncthreads();
@@ -564,10 +580,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) attention_decode_kernel(const 
         part[rr * (2 + kD) + 1] = l_run[rr];
     }
 #pragma unroll
-    for (int i = 0; i < kRows / 2; ++i) {
-        const int rr = half + 2 * i;
-        if (rr < p.rows) part[rr * (2 + kD) + 2 + d] = acc[i];
-    }
+    for (int i = 0; i < kRows; ++i)
+        if (i < p.rows) part[i * (2 + kD) + 2 + d] = acc[i];
 }
 
 template <int kRows>
@@ -580,35 +594,60 @@ cudaError_t launch_decode_rows(const DecodeParams &p, uint32_t smem, cudaStream_
                       s, p);
 }
 
-// Merges the chunks of one query row (a CTA of 128 threads, one per dimension).
-__global__ void __launch_bounds__(kD) attention_combine_kernel(const DecodeParams p) {
+// Merges the spans of one query row: 512 threads, four groups of 128 (one
+// thread per dimension) taking every fourth span, then a shared-memory sum.
+constexpr int kCombineGroups = 4;
+__global__ void __launch_bounds__(kD * kCombineGroups) attention_combine_kernel(const DecodeParams p) {
+    __shared__ float red[kD * kCombineGroups / 32];
+    __shared__ float part_acc[kCombineGroups - 1][kD];
+    __shared__ float part_l[kCombineGroups - 1];
     griddep_wait();
     griddep_launch_dependents();
-    const int rr = blockIdx.x, g = blockIdx.y, d = threadIdx.x;
+    const int rr = blockIdx.x, g = blockIdx.y, tid = threadIdx.x;
+    const int d = tid & (kD - 1), q = tid / kD;
     const int group = p.H / p.Hkv, hh = rr / p.m, t = rr % p.m;
     const float *base = p.part + static_cast<int64_t>(g) * p.n_chunks * p.rows * (2 + kD) + rr * (2 + kD);
     const int64_t step = static_cast<int64_t>(p.rows) * (2 + kD);
+    // the largest span maximum, over all 512 threads
     float mx = -INFINITY;
-#pragma unroll 8
-    for (int c = 0; c < p.n_chunks; ++c) mx = fmaxf(mx, base[c * step]);
+    for (int c = tid; c < p.n_chunks; c += kD * kCombineGroups) mx = fmaxf(mx, base[c * step]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+    if ((tid & 31) == 0) red[tid >> 5] = mx;
+    __syncthreads();
+    mx = red[0];
+#pragma unroll
+    for (int w = 1; w < kD * kCombineGroups / 32; ++w) mx = fmaxf(mx, red[w]);
     float l = 0.0f, acc = 0.0f;
 #pragma unroll 8
-    for (int c = 0; c < p.n_chunks; ++c) {
+    for (int c = q; c < p.n_chunks; c += kCombineGroups) {
         const float mc = base[c * step];
-        // a chunk with no visible key (maximum -inf) adds nothing
+        // a span with no visible key (maximum -inf) adds nothing
         const float f = mc == -INFINITY ? 0.0f : exp2f(mc - mx);
         l = fmaf(base[c * step + 1], f, l);
         acc = fmaf(base[c * step + 2 + d], f, acc);
     }
-    p.o[static_cast<int64_t>(t) * (p.H * kD) + (g * group + hh) * kD + d] = __float2bfloat16_rn(acc / l);
+    if (q > 0) {
+        part_acc[q - 1][d] = acc;
+        if (d == 0) part_l[q - 1] = l;
+    }
+    __syncthreads();
+    if (q == 0) {
+#pragma unroll
+        for (int i = 0; i < kCombineGroups - 1; ++i) {
+            acc += part_acc[i][d];
+            l += part_l[i];
+        }
+        p.o[static_cast<int64_t>(t) * (p.H * kD) + (g * group + hh) * kD + d] = __float2bfloat16_rn(acc / l);
+    }
 }
 
 }  // namespace
 
 size_t attention_decode_workspace_bytes(int64_t m, int64_t pos0, int64_t H, int64_t Hkv) {
-    // sized for one-sub-chunk spans, the most a launch uses on any GPU
     const int64_t rows = H / Hkv * m;
-    const int64_t n_chunks = (pos0 + m + kDecChunk - 1) / kDecChunk;
+    const int64_t span = kDecKeys * dec_span_blocks(pos0 + m, Hkv);
+    const int64_t n_chunks = (pos0 + m + span - 1) / span;
     return static_cast<size_t>(Hkv * n_chunks * rows * (2 + kD)) * sizeof(float);
 }
 
@@ -616,7 +655,7 @@ int attention_decode_max_rows() { return kDecMaxRows; }
 
 cudaError_t launch_attention_decode(const void *qkv, int64_t m, int64_t pos0, int64_t H, int64_t Hkv,
                                     void *k_cache, void *v_cache, int64_t S_max, void *o, void *ws,
-                                    int num_sms, cudaStream_t s) {
+                                    cudaStream_t s) {
     DecodeParams p;
     p.qkv = static_cast<const __nv_bfloat16 *>(qkv);
     p.k_cache = static_cast<__nv_bfloat16 *>(k_cache);
@@ -629,15 +668,16 @@ cudaError_t launch_attention_decode(const void *qkv, int64_t m, int64_t pos0, in
     p.Hkv = static_cast<int>(Hkv);
     p.S_max = static_cast<int>(S_max);
     p.rows = static_cast<int>(H / Hkv * m);
-    p.n_sub = dec_sub(p.rows, pos0 + m, Hkv, num_sms);
-    p.n_chunks = static_cast<int>((pos0 + m + kDecChunk * p.n_sub - 1) / (kDecChunk * p.n_sub));
+    p.span_blocks = static_cast<int>(dec_span_blocks(pos0 + m, Hkv));
+    const int64_t span = static_cast<int64_t>(kDecKeys) * p.span_blocks;
+    p.n_chunks = static_cast<int>((pos0 + m + span - 1) / span);
     cudaError_t e = launch_pdl(kv_append_kernel, dim3(p.m, p.Hkv), dim3(32), 0, s, p);
     if (e != cudaSuccess) return e;
     const uint32_t smem = kDecSmemFixed + kDecSmemPerRow * static_cast<uint32_t>(p.rows);
     e = p.rows <= 8 ? launch_decode_rows<8>(p, smem, s)
                     : (p.rows <= 32 ? launch_decode_rows<32>(p, smem, s) : launch_decode_rows<kDecMaxRows>(p, smem, s));
     if (e != cudaSuccess) return e;
-    e = launch_pdl(attention_combine_kernel, dim3(p.rows, p.Hkv), dim3(kD), 0, s, p);
+    e = launch_pdl(attention_combine_kernel, dim3(p.rows, p.Hkv), dim3(kD * kCombineGroups), 0, s, p);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 

@@ -751,7 +751,7 @@ mq_status mq_attention_decode_bf16(const void *qkv_bf16, int64_t m, int64_t pos0
     mq_status st = device_info(&d);
     if (st != MQ_OK) return st;
     return cuda_status(mq::launch_attention_decode(qkv_bf16, m, pos0, H, Hkv, k_cache, v_cache,
-                                                   S_max, o_bf16, workspace, d->num_sms, stream));
+                                                   S_max, o_bf16, workspace, stream));
 }
 
 mq_status mq_decode_linear_bf16(const mq_weight *w, const void *x_bf16, int64_t M, void *y_bf16,

@@ -117,7 +117,7 @@ int attention_decode_max_rows();
 // Appends the m new tokens' K / V to the cache, then the decode attention.
 cudaError_t launch_attention_decode(const void *qkv, int64_t m, int64_t pos0, int64_t H, int64_t Hkv,
                                     void *k_cache, void *v_cache, int64_t S_max, void *o, void *ws,
-                                    int num_sms, cudaStream_t s);
+                                    cudaStream_t s);
 
 // ---- decode (mq_decode.cu: BF16; mq_decode_nvf4.cu: NVFP4 W4A4) ----------------
 
