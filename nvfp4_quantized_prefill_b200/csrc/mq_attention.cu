@@ -387,26 +387,32 @@ EncodeFn encode_fn() {
 // Decode step: m new tokens at positions pos0 .. pos0 + m - 1.  Their K / V
 // rows are appended to the cache, then each query attends over keys
 // 0 .. pos0 + t of the cache.  Memory-bound (the cache is read once): the
-// keys are split into spans of 64-key blocks across many small CTAs (one CTA
-// per span and KV head, all of the group's query rows at once, so each K / V
-// byte crosses HBM once per step), each CTA leaves (max, sum, unnormalised o)
-// per query row, and a combine pass merges the spans.  FP32 throughout
-// (scores, weights, accumulation); BF16 output.
+// keys are split into spans across CTAs (one CTA per span and KV head, all of
+// the group's query rows at once, so each K / V byte crosses HBM once per
+// step); a CTA streams its span in 64-key blocks, double-buffered in shared
+// memory by cp.async, computes S = Q K^T and O += P V with BF16 m16n8k16
+// tensor-core MMAs (FP32 accumulation; P rounded to BF16 and the row sums
+// taken over the rounded weights, as in the prefill kernel), and leaves
+// (max, sum, unnormalised o) per query row; a combine pass merges the spans.
 
 constexpr int kDecKeys = 64;              // keys per block
-constexpr int kDecThreads = 128;          // 4 warps: 16 keys each for the scores, one dimension each for P.V
+constexpr int kDecThreads = 128;          // 4 warps: 16 keys each for S, 32 dimensions each for P.V
 constexpr int kDecMaxRows = 64;           // query rows per KV head (group size x tokens)
 #ifndef MQ_DEC_MAX_CTAS
-#define MQ_DEC_MAX_CTAS 2048
+#define MQ_DEC_MAX_CTAS 256
 #endif
-constexpr int kDecMaxCtas = MQ_DEC_MAX_CTAS;  // spans x KV heads stay below this (bounds the workspace)
-// shared memory: the block's V, then per query row its FP32 query and its
-// block of scores / weights (sized by the row count)
-constexpr uint32_t kDecSmemFixed = kDecKeys * kD * 2;
-constexpr uint32_t kDecSmemPerRow = kD * 4 + kDecKeys * 4;
+constexpr int kDecMaxCtas = MQ_DEC_MAX_CTAS;  // spans x KV heads stay at or below this
+constexpr uint32_t kDecTileBytes = kDecKeys * kD * 2;      // one K or V block, 16 KB
+constexpr int kDecQPitch = kD + 8;                          // BF16 per Q row (bank-conflict-free)
+constexpr int kDecPPitch = kDecKeys + 8;                    // BF16 per P row
+// shared memory: K and V blocks (two each), then Q, P and the per-warp row
+// maxima / sums for kNT row tiles of 8
+template <int kNT>
+constexpr uint32_t dec_smem_bytes() {
+    return 4 * kDecTileBytes + 8 * kNT * (kDecQPitch * 2 + kDecPPitch * 2 + 2 * 4 * 4);
+}
 
-// 64-key blocks per span: one, unless the cache is long enough that the
-// spans x KV heads would pass kDecMaxCtas
+// 64-key blocks per span: as few as keep spans x KV heads within kDecMaxCtas
 __host__ __device__ constexpr int64_t dec_span_blocks(int64_t n_keys, int64_t Hkv) {
     const int64_t blocks = (n_keys + kDecKeys - 1) / kDecKeys;
     const int64_t sb = (blocks * Hkv + kDecMaxCtas - 1) / kDecMaxCtas;
@@ -440,158 +446,250 @@ __global__ void __launch_bounds__(32) kv_append_kernel(const DecodeParams p) {
         reinterpret_cast<uint4 *>(p.v_cache + dst)[lane - 16] = src_v[lane - 16];
 }
 
-__device__ __forceinline__ uint4 ldg_nc_v4(const void *ptr) {
-    uint4 v;
-    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(ptr));
-    return v;
-}
-
 // 16 bytes global -> shared, asynchronously; src_bytes = 0 fills zeros
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
                  : "memory");
 }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+// D (16x8 FP32) += A (16x16 BF16, row-major) * B (16x8 BF16, column-major)
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// kRows: the largest query-row count this instance serves (its share of o in
-// registers scales with it)
-template <int kRows>
+// byte offset of (key, 8-element chunk c) in a [64][128] BF16 block whose
+// 16-byte chunks are XOR-swizzled by the key's low three bits
+__device__ __forceinline__ uint32_t dec_tile_off(int key, int c) {
+    return static_cast<uint32_t>(key * 256 + ((c ^ (key & 7)) << 4));
+}
+
+// kNT: 8-row tiles of query rows this instance serves (rows <= 8 kNT)
+template <int kNT>
 __global__ void __launch_bounds__(kDecThreads) attention_decode_kernel(const DecodeParams p) {
-    extern __shared__ __align__(16) uint8_t dsm[];
-    __nv_bfloat16 *vs = reinterpret_cast<__nv_bfloat16 *>(dsm);                        // [64][128]
-    float *qs = reinterpret_cast<float *>(dsm + kDecSmemFixed);                          // [rows][128]
-    float *ps = qs + p.rows * kD;                                                        // [rows][64]
+    extern __shared__ __align__(128) uint8_t dsm[];
+    const uint32_t kv0 = smem_u32(dsm);                     // K[2], V[2]: 4 x 16 KB
+    __nv_bfloat16 *qs = reinterpret_cast<__nv_bfloat16 *>(dsm + 4 * kDecTileBytes);   // [8 kNT][136]
+    __nv_bfloat16 *ps = qs + 8 * kNT * kDecQPitch;                                     // [8 kNT][72]
+    float *red_max = reinterpret_cast<float *>(ps + 8 * kNT * kDecPPitch);             // [4][8 kNT]
+    float *red_sum = red_max + 4 * 8 * kNT;                                             // [4][8 kNT]
     __shared__ float m_run[kDecMaxRows], l_run[kDecMaxRows], alpha[kDecMaxRows];
     const int c = blockIdx.x, g = blockIdx.y, tid = threadIdx.x;
-    const int warp = tid >> 5, lane = tid & 31;
+    const int warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
     const int group = p.H / p.Hkv;
     const int n_keys = p.pos0 + p.m;
     const int cols = (p.H + 2 * p.Hkv) * kD;
     const __nv_bfloat16 *kbase = p.k_cache + static_cast<int64_t>(g) * p.S_max * kD;
     const __nv_bfloat16 *vbase = p.v_cache + static_cast<int64_t>(g) * p.S_max * kD;
-    const uint32_t vs_addr = smem_u32(vs);
+    const int key_begin = c * p.span_blocks * kDecKeys;
+    const int nb = min(p.span_blocks, (n_keys - key_begin + kDecKeys - 1) / kDecKeys);
+    // block b of the span into buffer b & 1 (K at kv0 + buf 16 KB, V two buffers on)
+    auto load_block = [&](int b) {
+        const int key0 = key_begin + b * kDecKeys;
+        const uint32_t kdst = kv0 + static_cast<uint32_t>(b & 1) * kDecTileBytes;
+        const uint32_t vdst = kdst + 2 * kDecTileBytes;
+        for (int i = tid; i < kDecKeys * (kD / 8); i += kDecThreads) {
+            const int k = i >> 4, ch = i & 15;
+            const bool in = key0 + k < n_keys;
+            const int64_t off = static_cast<int64_t>(in ? key0 + k : key0) * kD + ch * 8;
+            cp_async16(kdst + dec_tile_off(k, ch), kbase + off, in ? 16u : 0u);
+            cp_async16(vdst + dec_tile_off(k, ch), vbase + off, in ? 16u : 0u);
+        }
+        cp_async_commit();
+    };
     griddep_wait();            // the appended rows and the queries are in place
     griddep_launch_dependents();
-    // the group's query rows: row rr = hh * m + t (head g * group + hh, token t)
-    for (int i = tid; i < p.rows * kD; i += kDecThreads) {
-        const int rr = i / kD, d = i % kD, hh = rr / p.m, t = rr % p.m;
-        qs[rr * kD + d] = __bfloat162float(p.qkv[static_cast<int64_t>(t) * cols + (g * group + hh) * kD + d]);
+    load_block(0);
+    // the group's query rows (row rr = hh * m + t: head g * group + hh, token t), zeros past p.rows
+    for (int i = tid; i < 8 * kNT * (kD / 2); i += kDecThreads) {
+        const int rr = i / (kD / 2), d2 = (i % (kD / 2)) * 2;
+        uint32_t v = 0;
+        if (rr < p.rows) {
+            const int hh = rr / p.m, t = rr % p.m;
+            v = *reinterpret_cast<const uint32_t *>(p.qkv + static_cast<int64_t>(t) * cols + (g * group + hh) * kD + d2);
+        }
+        *reinterpret_cast<uint32_t *>(qs + rr * kDecQPitch + d2) = v;
     }
-    for (int rr = tid; rr < p.rows; rr += kDecThreads) {
+    for (int rr = tid; rr < kDecMaxRows; rr += kDecThreads) {
         m_run[rr] = -INFINITY;
         l_run[rr] = 0.0f;
     }
-    // scores: this lane takes key kk of the block, dimensions [64 kh, 64 kh + 64)
-    const int kk = warp * 16 + (lane & 15), kh = lane >> 4;
-    // P.V: this thread's dimension of every row
-    const int d = tid;
-    float acc[kRows];
+    // P.V accumulators: dims 32 warp + 16 i + gq (+ 8), rows 8 j + 2 tq (+ 1)
+    float acc[2][kNT][4];
 #pragma unroll
-    for (int i = 0; i < kRows; ++i) acc[i] = 0.0f;
-    for (int b = 0; b < p.span_blocks; ++b) {
-        const int key0 = (c * p.span_blocks + b) * kDecKeys;
-        if (key0 >= n_keys) break;   // uniform over the CTA
-        const int nk = min(kDecKeys, n_keys - key0);
-        __syncthreads();             // the previous block's V and weights are consumed
-        // this lane's half key row into registers (zeros past the cache's end)
-        uint32_t kr[32];
-        {
-            const int key = kk < nk ? key0 + kk : key0;
-            const uint4 *src = reinterpret_cast<const uint4 *>(kbase + static_cast<int64_t>(key) * kD + kh * 64);
+    for (int i = 0; i < 2; ++i)
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                uint4 v = ldg_nc_v4(src + j);
-                if (kk >= nk) v = make_uint4(0, 0, 0, 0);
-                kr[4 * j] = v.x; kr[4 * j + 1] = v.y; kr[4 * j + 2] = v.z; kr[4 * j + 3] = v.w;
+        for (int j = 0; j < kNT; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.0f;
+    for (int b = 0; b < nb; ++b) {
+        if (b + 1 < nb) {
+            load_block(b + 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();           // block b (and, the first time, Q) is in shared memory
+        const int key0 = key_begin + b * kDecKeys;
+        const uint32_t kt = kv0 + static_cast<uint32_t>(b & 1) * kDecTileBytes;
+        const uint32_t vt = kt + 2 * kDecTileBytes;
+        // S^T (keys 16 warp .. of the block x rows) = K Q^T
+        float sc[kNT][4];
+#pragma unroll
+        for (int j = 0; j < kNT; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sc[j][e] = 0.0f;
+#pragma unroll
+        for (int s = 0; s < kD / 16; ++s) {
+            uint32_t a[4];
+            ldsm_x4(kt + dec_tile_off(16 * warp + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * s + (lane >> 4)), a);
+#pragma unroll
+            for (int j = 0; j < kNT; ++j) {
+                const __nv_bfloat16 *qr = qs + (8 * j + gq) * kDecQPitch + 16 * s + 2 * tq;
+                mma_bf16_16816(sc[j], a, *reinterpret_cast<const uint32_t *>(qr),
+                               *reinterpret_cast<const uint32_t *>(qr + 8));
             }
         }
-        // the block's V into shared memory, asynchronously (zeros past the end)
-        for (int i = tid; i < kDecKeys * (kD / 8); i += kDecThreads) {
-            const int k = i >> 4, c16 = i & 15;
-            const int key = k < nk ? key0 + k : key0;
-            cp_async16(vs_addr + static_cast<uint32_t>(i) * 16u, vbase + static_cast<int64_t>(key) * kD + c16 * 8,
-                       k < nk ? 16u : 0u);
-        }
-        // scores in the base-2 exponent domain; masked: past the cache or
-        // after the row's own position
-        const int pos = key0 + kk;
-        for (int r = 0; r < p.rows; ++r) {
-            const float *q = qs + r * kD + kh * 64;
-            float a0 = 0.0f, a1 = 0.0f;
+        // scale, mask (past the cache, after the row's own position, padding
+        // rows), and the block maximum of each row over this warp's keys
+        float mx[kNT][2];
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-                const float4 qv = *reinterpret_cast<const float4 *>(q + 2 * j);
-                a0 = fmaf(qv.x, __uint_as_float(kr[j] << 16), a0);
-                a1 = fmaf(qv.y, __uint_as_float(kr[j] & 0xFFFF0000u), a1);
-                a0 = fmaf(qv.z, __uint_as_float(kr[j + 1] << 16), a0);
-                a1 = fmaf(qv.w, __uint_as_float(kr[j + 1] & 0xFFFF0000u), a1);
+        for (int j = 0; j < kNT; ++j) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int row = 8 * j + 2 * tq + (e & 1);
+                const int pos = key0 + 16 * warp + gq + (e >> 1) * 8;
+                const bool ok = row < p.rows && pos < n_keys && pos <= p.pos0 + row % p.m;
+                sc[j][e] = ok ? sc[j][e] * kScaleLog2 : -INFINITY;
             }
-            float sc = a0 + a1;
-            sc += __shfl_xor_sync(0xFFFFFFFFu, sc, 16);
-            const int t = r % p.m;
-            if (lane < 16) ps[r * kDecKeys + kk] = (kk < nk && pos <= p.pos0 + t) ? sc * kScaleLog2 : -INFINITY;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float v = fmaxf(sc[j][h], sc[j][h + 2]);
+#pragma unroll
+                for (int o = 4; o < 32; o <<= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+                mx[j][h] = v;
+            }
+            if (gq == 0) {
+                red_max[warp * 8 * kNT + 8 * j + 2 * tq] = mx[j][0];
+                red_max[warp * 8 * kNT + 8 * j + 2 * tq + 1] = mx[j][1];
+            }
         }
         __syncthreads();
-        // per row: running maximum, weights 2^(x - max), running sum (a warp a row)
-        for (int r = warp; r < p.rows; r += kDecThreads / 32) {
-            const float x0 = ps[r * kDecKeys + lane], x1 = ps[r * kDecKeys + lane + 32];
-            float mx = fmaxf(x0, x1);
+        // weights 2^(s - m_new) rounded to BF16 (the P.V operand), and their row sums
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-            const float m_old = m_run[r];
-            const float m_new = fmaxf(m_old, mx);
-            const float w0 = m_new == -INFINITY ? 0.0f : exp2f(x0 - m_new);
-            const float w1 = m_new == -INFINITY ? 0.0f : exp2f(x1 - m_new);
-            ps[r * kDecKeys + lane] = w0;
-            ps[r * kDecKeys + lane + 32] = w1;
-            float sum = w0 + w1;
+        for (int j = 0; j < kNT; ++j) {
+            float mnew[2], sum[2];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
-            if (lane == 0) {
-                const float a = (m_old == -INFINITY) ? 0.0f : exp2f(m_old - m_new);
-                alpha[r] = a;
-                l_run[r] = l_run[r] * a + sum;
-                m_run[r] = m_new;
+            for (int h = 0; h < 2; ++h) {
+                const int row = 8 * j + 2 * tq + h;
+                float v = m_run[row];
+#pragma unroll
+                for (int w = 0; w < 4; ++w) v = fmaxf(v, red_max[w * 8 * kNT + row]);
+                mnew[h] = v;
+                sum[h] = 0.0f;
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int h = e & 1;
+                const float w = mnew[h] == -INFINITY ? 0.0f : exp2f(sc[j][e] - mnew[h]);
+                const __nv_bfloat16 wb = __float2bfloat16_rn(w);
+                sum[h] += __bfloat162float(wb);
+                ps[(8 * j + 2 * tq + h) * kDecPPitch + 16 * warp + gq + (e >> 1) * 8] = wb;
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float v = sum[h];
+#pragma unroll
+                for (int o = 4; o < 32; o <<= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+                if (gq == 0) red_sum[warp * 8 * kNT + 8 * j + 2 * tq + h] = v;
             }
         }
-        cp_async_wait_all();
         __syncthreads();
-        // o: rescale, then add the block's weighted values (each value read
-        // once for all rows; the weights are broadcast)
+        // running maximum and sum per row
+        for (int row = tid; row < 8 * kNT; row += kDecThreads) {
+            float v = m_run[row];
 #pragma unroll
-        for (int i = 0; i < kRows; ++i)
-            if (i < p.rows) acc[i] *= alpha[i];
-        for (int k = 0; k < nk; ++k) {
-            const float v = __bfloat162float(vs[k * kD + d]);
+            for (int w = 0; w < 4; ++w) v = fmaxf(v, red_max[w * 8 * kNT + row]);
+            const float m_old = m_run[row];
+            const float a = m_old == -INFINITY ? 0.0f : exp2f(m_old - v);
+            float l = 0.0f;
 #pragma unroll
-            for (int i = 0; i < kRows; ++i)
-                if (i < p.rows) acc[i] = fmaf(ps[i * kDecKeys + k], v, acc[i]);
+            for (int w = 0; w < 4; ++w) l += red_sum[w * 8 * kNT + row];
+            alpha[row] = a;
+            l_run[row] = l_run[row] * a + l;
+            m_run[row] = v;
         }
+        __syncthreads();
+        // O^T (dims x rows) = alpha O^T + V^T P^T over the block's 64 keys
+#pragma unroll
+        for (int j = 0; j < kNT; ++j) {
+            const float a0 = alpha[8 * j + 2 * tq], a1 = alpha[8 * j + 2 * tq + 1];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                acc[i][j][0] *= a0;
+                acc[i][j][1] *= a1;
+                acc[i][j][2] *= a0;
+                acc[i][j][3] *= a1;
+            }
+        }
+#pragma unroll
+        for (int s = 0; s < kDecKeys / 16; ++s) {
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                uint32_t a[4];
+                const int mi = lane >> 3;
+                ldsm_x4_trans(vt + dec_tile_off(16 * s + (lane & 7) + (mi >> 1) * 8, 4 * warp + 2 * i + (mi & 1)), a);
+#pragma unroll
+                for (int j = 0; j < kNT; ++j) {
+                    const __nv_bfloat16 *pr = ps + (8 * j + gq) * kDecPPitch + 16 * s + 2 * tq;
+                    mma_bf16_16816(acc[i][j], a, *reinterpret_cast<const uint32_t *>(pr),
+                                   *reinterpret_cast<const uint32_t *>(pr + 8));
+                }
+            }
+        }
+        __syncthreads();           // buffers b & 1, P and the row partials may be overwritten
     }
-    __syncthreads();
     float *part = p.part + (static_cast<int64_t>(g) * p.n_chunks + c) * p.rows * (2 + kD);
     for (int rr = tid; rr < p.rows; rr += kDecThreads) {
         part[rr * (2 + kD)] = m_run[rr];
         part[rr * (2 + kD) + 1] = l_run[rr];
     }
 #pragma unroll
-    for (int i = 0; i < kRows; ++i)
-        if (i < p.rows) part[i * (2 + kD) + 2 + d] = acc[i];
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < kNT; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int row = 8 * j + 2 * tq + (e & 1);
+                const int d = 32 * warp + 16 * i + gq + (e >> 1) * 8;
+                if (row < p.rows) part[row * (2 + kD) + 2 + d] = acc[i][j][e];
+            }
 }
 
-template <int kRows>
-cudaError_t launch_decode_rows(const DecodeParams &p, uint32_t smem, cudaStream_t s) {
-    cudaError_t e = cudaFuncSetAttribute(attention_decode_kernel<kRows>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kDecSmemFixed + kDecSmemPerRow * kRows);
+template <int kNT>
+cudaError_t launch_decode_rows(const DecodeParams &p, cudaStream_t s) {
+    constexpr uint32_t smem = dec_smem_bytes<kNT>();
+    cudaError_t e = cudaFuncSetAttribute(attention_decode_kernel<kNT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(attention_decode_kernel<kRows>, dim3(p.n_chunks, p.Hkv), dim3(kDecThreads), smem,
-                      s, p);
+    return launch_pdl(attention_decode_kernel<kNT>, dim3(p.n_chunks, p.Hkv), dim3(kDecThreads), smem, s, p);
 }
 
 // Merges the spans of one query row: 512 threads, four groups of 128 (one
@@ -673,9 +771,8 @@ cudaError_t launch_attention_decode(const void *qkv, int64_t m, int64_t pos0, in
     p.n_chunks = static_cast<int>((pos0 + m + span - 1) / span);
     cudaError_t e = launch_pdl(kv_append_kernel, dim3(p.m, p.Hkv), dim3(32), 0, s, p);
     if (e != cudaSuccess) return e;
-    const uint32_t smem = kDecSmemFixed + kDecSmemPerRow * static_cast<uint32_t>(p.rows);
-    e = p.rows <= 8 ? launch_decode_rows<8>(p, smem, s)
-                    : (p.rows <= 32 ? launch_decode_rows<32>(p, smem, s) : launch_decode_rows<kDecMaxRows>(p, smem, s));
+    e = p.rows <= 8 ? launch_decode_rows<1>(p, s)
+                    : (p.rows <= 32 ? launch_decode_rows<4>(p, s) : launch_decode_rows<kDecMaxRows / 8>(p, s));
     if (e != cudaSuccess) return e;
     e = launch_pdl(attention_combine_kernel, dim3(p.rows, p.Hkv), dim3(kD * kCombineGroups), 0, s, p);
     return e != cudaSuccess ? e : cudaGetLastError();
