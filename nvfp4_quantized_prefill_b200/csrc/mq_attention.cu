@@ -43,11 +43,18 @@ constexpr uint32_t kQOff = 0;
 constexpr uint32_t kKOff = kTileBytes;                       // K stages
 constexpr uint32_t kVOff = kKOff + kStages * kTileBytes;     // V stages
 constexpr uint32_t kBarOff = kVOff + kStages * kTileBytes;
-constexpr uint32_t kXchgOff = kBarOff + 256;                 // row maxima, 2 tiles x 2 halves x 128
-constexpr uint32_t kLsumOff = kXchgOff + 2 * 2 * 128 * 4;    // row sums, 2 halves x 128
-constexpr uint32_t kSmemBytes = kLsumOff + 2 * 128 * 4 + 1024;
-constexpr int kSoftmaxWarps = 8;          // two warpgroups: columns 0-63 and 64-127 of every row
-constexpr int kThreads = 32 * (2 + kSoftmaxWarps);   // producer, MMA, softmax
+#ifndef MQ_ATT_COL_GROUPS
+#define MQ_ATT_COL_GROUPS 2
+#endif
+constexpr int kColGroups = MQ_ATT_COL_GROUPS;   // softmax warpgroups, each a column range of every row
+constexpr int kCols = 128 / kColGroups;          // S columns per softmax thread
+constexpr uint32_t kXchgOff = kBarOff + 256;     // row maxima, 2 tiles x kColGroups x 128
+constexpr uint32_t kLsumOff = kXchgOff + 2 * kColGroups * 128 * 4;   // row sums, kColGroups x 128
+constexpr uint32_t kSmemBytes = kLsumOff + kColGroups * 128 * 4 + 1024;
+constexpr int kSoftmaxWarps = 4 * kColGroups;
+static_assert(kCols % 32 == 0, "whole 32-column TMEM loads per thread");
+constexpr int kSoftWarp0 = 3;             // warps 0-2: producer, S issuer, PV issuer
+constexpr int kThreads = 32 * (kSoftWarp0 + kSoftmaxWarps);
 constexpr int kSBufs = 3;                 // S / P buffers in tensor memory
 constexpr uint32_t kTmemCols = 512;       // S0, S1, S2 at 0, 128, 256; O at 384
 constexpr uint32_t kOCol = 128 * kSBufs;
@@ -63,6 +70,14 @@ struct PrefillParams {
     int partial_slots;        // > 0: atomicMax into amax_partials[cta % slots]
     unsigned *err;
 };
+
+// 2^x by the hardware approximation (relative error about 2^-22, subnormal
+// results flushed to zero): the weights it feeds are rounded to BF16.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 // Bounded wait on an mbarrier phase (all lanes poll); false after the limit.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity) {
@@ -85,15 +100,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t q_full = bar;
     const uint32_t k_full = bar + 8;          // [2] per K/V stage
     const uint32_t v_full = bar + 24;         // [2]
-    const uint32_t kv_empty = bar + 40;       // [2]
+    const uint32_t k_empty = bar + 40;        // [2] S of that stage's K tile has completed
+    const uint32_t v_empty = bar + 232;       // [2] PV of that stage's V tile has completed
     const uint32_t s_full = bar + 56;         // [3] per S buffer
     const uint32_t p_full = bar + 80;         // [3]
     const uint32_t pv_done = bar + 104;       // [3] the PV product that read P of that buffer
     const uint32_t drain = bar + 128;         // every MMA issued has completed
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kBarOff + 136);
-    float *red = reinterpret_cast<float *>(smem + kBarOff + 160);   // 8 floats
-    float *xchg = reinterpret_cast<float *>(smem + kXchgOff);      // [2][2][128]
-    float *lsum = reinterpret_cast<float *>(smem + kLsumOff);      // [2][128]
+    float *red = reinterpret_cast<float *>(smem + kBarOff + 160);   // one float per softmax warp
+    float *xchg = reinterpret_cast<float *>(smem + kXchgOff);      // [2][kColGroups][128]
+    float *lsum = reinterpret_cast<float *>(smem + kLsumOff);      // [kColGroups][128]
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -111,14 +127,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < kStages; ++i) {
             mbar_init(k_full + 8 * i, 1);
             mbar_init(v_full + 8 * i, 1);
-            mbar_init(kv_empty + 8 * i, 1);
+            mbar_init(k_empty + 8 * i, 1);
+            mbar_init(v_empty + 8 * i, 1);
         }
         for (int i = 0; i < kSBufs; ++i) {
             mbar_init(s_full + 8 * i, 1);
             mbar_init(p_full + 8 * i, kSoftmaxWarps);   // one arrival per softmax warp
             mbar_init(pv_done + 8 * i, 1);
         }
-        mbar_init(drain, 1);
+        mbar_init(drain, 2);                       // one commit per MMA-issuing warp
         fence_barrier_init();
         prefetch_tmap(&tmap_qkv);
         if (p.write_cache) {
@@ -143,20 +160,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d(s0 + kQOff + kHalfBytes, &tmap_qkv, qkv_cols_q + 64, qt * kTile, q_full);
             const bool writer = p.write_cache && (h % group) == 0;
             bool stored[kStages] = {false, false};
+            int last_k = -1, last_v = -1;   // the last tiles whose K / V loads were issued
             for (int j = 0; j < nkv && ok; ++j) {
                 const int st = j & 1;
-                if (j >= kStages) {
-                    if (!wait_bar(kv_empty + 8 * st, ((j - kStages) >> 1) & 1)) ok = false;
-                    if (stored[st]) {
-                        bulk_wait_group_read0();   // the cache store has read the stage
-                        stored[st] = false;
-                    }
+                // K and V tiles are released separately (K once S has read it,
+                // V once PV has), so the next K tile does not wait for a softmax;
+                // a barrier is re-armed only after its previous phase completed
+                if (j >= kStages && !wait_bar(k_empty + 8 * st, ((j - kStages) >> 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                if (stored[st]) {
+                    bulk_wait_group_read0();   // the cache store has read the stage
+                    stored[st] = false;
                 }
                 const uint32_t ks = s0 + kKOff + st * kTileBytes;
                 const uint32_t vs = s0 + kVOff + st * kTileBytes;
                 mbar_arrive_expect_tx(k_full + 8 * st, kTileBytes);
                 tma_load_2d(ks, &tmap_qkv, qkv_cols_k, j * kTile, k_full + 8 * st);
                 tma_load_2d(ks + kHalfBytes, &tmap_qkv, qkv_cols_k + 64, j * kTile, k_full + 8 * st);
+                if (j >= kStages && !wait_bar(v_empty + 8 * st, ((j - kStages) >> 1) & 1)) {
+                    ok = false;
+                    last_k = j;
+                    break;
+                }
+                last_k = last_v = j;
                 mbar_arrive_expect_tx(v_full + 8 * st, kTileBytes);
                 tma_load_2d(vs, &tmap_qkv, qkv_cols_v, j * kTile, v_full + 8 * st);
                 tma_load_2d(vs + kHalfBytes, &tmap_qkv, qkv_cols_v + 64, j * kTile, v_full + 8 * st);
@@ -174,102 +202,118 @@ __global__ void __launch_bounds__(kThreads, 1)
                     stored[st] = true;
                 }
             }
-            // the loads of the last tile of each stage have landed (they have on
-            // the normal path; after a timeout, before the CTA may exit)
-            for (int j = nkv - 1; j >= 0 && j >= nkv - kStages; --j) {
-                wait_bar(k_full + 8 * (j & 1), (j >> 1) & 1);
-                wait_bar(v_full + 8 * (j & 1), (j >> 1) & 1);
-            }
+            // the loads of the last tiles of each stage have landed (they have
+            // on the normal path; after a timeout, before the CTA may exit)
+            for (int j = last_k; j >= 0 && j > last_k - kStages; --j) wait_bar(k_full + 8 * (j & 1), (j >> 1) & 1);
+            for (int j = last_v; j >= 0 && j > last_v - kStages; --j) wait_bar(v_full + 8 * (j & 1), (j >> 1) & 1);
             bulk_wait_group0();   // cache stores complete before the CTA exits
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------------------------------------------------- MMA issuer
+        // ---------------------------------------------------------- S = Q K^T issuer
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16(128, 128, 0, 0);   // Q, K both K-major
-            constexpr uint32_t idesc_o = idesc_bf16(128, 128, 0, 1);   // V MN-major
             if (!wait_bar(q_full, 0)) ok = false;
             tc_fence_after();
-            for (int j = 0; j <= nkv && ok; ++j) {
-                if (j < nkv) {
-                    const int st = j & 1, sb = j % kSBufs;
-                    if (!wait_bar(k_full + 8 * st, (j >> 1) & 1)) ok = false;
-                    // S buffer sb last held P_{j-3}: its PV must have completed
-                    if (j >= kSBufs && !wait_bar(pv_done + 8 * sb, ((j - kSBufs) / kSBufs) & 1)) ok = false;
-                    tc_fence_after();
-                    tc_mma8_bf16_ss_commit(tmem + sb * 128u, sdesc_kmajor_sw128(s0 + kQOff),
-                                           sdesc_kmajor_sw128(s0 + kKOff + st * kTileBytes), idesc_s, 0u,
-                                           s_full + 8 * sb);
-                }
-                if (j >= 1) {
-                    const int jj = j - 1, st = jj & 1, sb = jj % kSBufs;
-                    if (!wait_bar(p_full + 8 * sb, (jj / kSBufs) & 1)) ok = false;
-                    if (!wait_bar(v_full + 8 * st, (jj >> 1) & 1)) ok = false;
-                    tc_fence_after();
-                    // keys 16 kk .. 16 kk + 15: two 8-row groups of the V tile
-                    tc_mma8_bf16_ts_commit2(tmem + kOCol, tmem + sb * 128u,
-                                            sdesc_mnmajor_sw128(s0 + kVOff + st * kTileBytes, kHalfBytes),
-                                            idesc_o, jj > 0 ? 1u : 0u, pv_done + 8 * sb,
-                                            kv_empty + 8 * st);
-                }
+            for (int j = 0; j < nkv && ok; ++j) {
+                const int st = j & 1, sb = j % kSBufs;
+                if (!wait_bar(k_full + 8 * st, (j >> 1) & 1)) ok = false;
+                // S buffer sb last held P_{j-3}: its PV must have completed
+                if (j >= kSBufs && !wait_bar(pv_done + 8 * sb, ((j - kSBufs) / kSBufs) & 1)) ok = false;
+                if (!ok) break;
+                tc_fence_after();
+                tc_mma8_bf16_ss_commit2(tmem + sb * 128u, sdesc_kmajor_sw128(s0 + kQOff),
+                                        sdesc_kmajor_sw128(s0 + kKOff + st * kTileBytes), idesc_s, 0u,
+                                        s_full + 8 * sb, k_empty + 8 * st);
             }
             // every MMA this thread issued completes before TMEM is freed
             tc_commit(drain);
             wait_bar(drain, 0);
         }
         __syncwarp();
+    } else if (warp == 2) {
+        // ---------------------------------------------------------- O += P V issuer
+        // (its own warp: the two products of a tile go to different TMEM
+        // regions and are ordered only through the barriers, so S of later
+        // tiles is issued while this warp waits for a softmax)
+        if (lane == 0) {
+            constexpr uint32_t idesc_o = idesc_bf16(128, 128, 0, 1);   // V MN-major
+            for (int jj = 0; jj < nkv && ok; ++jj) {
+                const int st = jj & 1, sb = jj % kSBufs;
+                if (!wait_bar(p_full + 8 * sb, (jj / kSBufs) & 1)) ok = false;
+                if (!wait_bar(v_full + 8 * st, (jj >> 1) & 1)) ok = false;
+                if (!ok) break;
+                tc_fence_after();
+                // keys 16 kk .. 16 kk + 15: two 8-row groups of the V tile
+                tc_mma8_bf16_ts_commit2(tmem + kOCol, tmem + sb * 128u,
+                                        sdesc_mnmajor_sw128(s0 + kVOff + st * kTileBytes, kHalfBytes),
+                                        idesc_o, jj > 0 ? 1u : 0u, pv_done + 8 * sb, v_empty + 8 * st);
+            }
+            tc_commit(drain);
+            wait_bar(drain, 0);
+        }
+        __syncwarp();
     } else {
         // ---------------------------------------------------------- softmax
-        // warpgroup wg holds columns [64 wg, 64 wg + 64) of every row; the two
-        // threads of a row agree on the row maximum through shared memory
-        // (one named barrier a tile, double-buffered by tile parity) and keep
-        // their own share of the row sum
-        const int wg = (warp - 2) >> 2;
+        // warpgroup wg holds columns [kCols wg, kCols wg + kCols) of every row;
+        // the kColGroups threads of a row agree on the row maximum through
+        // shared memory (one named barrier a tile, double-buffered by tile
+        // parity) and keep their own share of the row sum
+        const int wg = (warp - kSoftWarp0) >> 2;
         const int quarter = warp & 3;             // TMEM lane group of this warp
         const int r = quarter * 32 + lane;        // query row in the tile
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-        const int col0 = wg * 64;
+        const int col0 = wg * kCols;
         float m_run = -INFINITY, l = 0.0f;
         for (int j = 0; j < nkv; ++j) {
             const int st = j & 1, sb = j % kSBufs;
             ok = __all_sync(0xFFFFFFFFu, wait_bar(s_full + 8 * sb, (j / kSBufs) & 1)) && ok;
             tc_fence_after();
-            uint32_t sr[64];
-            tmem_ld32(tmem + lane_off + sb * 128u + col0, *reinterpret_cast<uint32_t (*)[32]>(&sr[0]));
-            tmem_ld32(tmem + lane_off + sb * 128u + col0 + 32u, *reinterpret_cast<uint32_t (*)[32]>(&sr[32]));
+            uint32_t sr[kCols];
+#pragma unroll
+            for (int h = 0; h < kCols / 32; ++h)
+                tmem_ld32(tmem + lane_off + sb * 128u + col0 + 32u * h,
+                          *reinterpret_cast<uint32_t (*)[32]>(&sr[32 * h]));
             tmem_ld_wait();
-            float s[64];
+            // raw scores (the base-2 scale is applied inside the exponent);
+            // keys after the row's own position masked on the diagonal tile
+            float s[kCols];
+#pragma unroll
+            for (int c = 0; c < kCols; ++c) s[c] = __uint_as_float(sr[c]);
+            if (j == qt) {
+#pragma unroll
+                for (int c = 0; c < kCols; ++c)
+                    if (col0 + c > r) s[c] = -INFINITY;
+            }
             float mp[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) mp[e] = -INFINITY;
-            const bool diag = (j == qt);
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                float x = __uint_as_float(sr[c]) * kScaleLog2;
-                if (diag && col0 + c > r) x = -INFINITY;
-                s[c] = x;
-                mp[c & 7] = fmaxf(mp[c & 7], x);   // eight independent chains
-            }
+            for (int c = 0; c < kCols; ++c) mp[c & 7] = fmaxf(mp[c & 7], s[c]);   // eight chains
+            // the scale is positive: the maximum of the scaled scores
             float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-            xchg[(st * 2 + wg) * 128 + r] = mx;
+                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) * kScaleLog2;
+            xchg[(st * kColGroups + wg) * 128 + r] = mx;
             // the barrier's AND also carries "every softmax warp saw S": after
-            // a timed-out wait all eight warps leave the loop together (none
-            // may be left waiting here for the others)
+            // a timed-out wait all softmax warps leave the loop together (none
+            // may be left waiting here for the others); it also orders every
+            // thread's S loads before any thread's P stores over the buffer
             uint32_t all_ok;
             asm volatile(
                 "{\n\t.reg .pred p, q;\n\t"
                 "setp.ne.u32 p, %1, 0;\n\t"
-                "bar.red.and.pred q, 2, 256, p;\n\t"
+                "bar.red.and.pred q, 2, %2, p;\n\t"
                 "selp.u32 %0, 1, 0, q;\n\t}"
                 : "=r"(all_ok)
-                : "r"(ok ? 1u : 0u)
+                : "r"(ok ? 1u : 0u), "n"(32 * kSoftmaxWarps)
                 : "memory");
             if (!all_ok) {
                 ok = false;
                 break;
             }
-            mx = fmaxf(mx, xchg[(st * 2 + (1 - wg)) * 128 + r]);
+#pragma unroll
+            for (int w2 = 0; w2 < kColGroups; ++w2)
+                if (w2 != wg) mx = fmaxf(mx, xchg[(st * kColGroups + w2) * 128 + r]);
             // raise the running maximum only for a growth beyond 2^8 (or at
             // the first tile); O then needs the factor 2^(m_old - m_new)
             const bool need = mx > m_run + kRescaleThreshold;
@@ -282,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 wait_bar(pv_done + 8 * ((j - 1) % kSBufs), ((j - 1) / kSBufs) & 1)) && ok;
                 tc_fence_after();
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
+                for (int c = 0; c < kCols / 32; ++c) {
                     uint32_t ov[32];
                     tmem_ld32(tmem + lane_off + kOCol + col0 + c * 32u, ov);
                     tmem_ld_wait();
@@ -294,27 +338,36 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             l *= f;
             m_run = m_new;
-            uint32_t pk[32];
+            const float neg_m = -m_run;
             float lp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const __nv_bfloat162 pb =
-                    __floats2bfloat162_rn(exp2f(s[2 * c] - m_run), exp2f(s[2 * c + 1] - m_run));
-                // the row sum of the BF16 weights the PV product uses
-                lp[c & 3] += __bfloat162float(pb.x) + __bfloat162float(pb.y);
-                pk[c] = *reinterpret_cast<const uint32_t *>(&pb);
+            for (int h = 0; h < kCols / 32; ++h) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    const int cc = 16 * h + c;
+                    const __nv_bfloat162 pb =
+                        __floats2bfloat162_rn(ex2_approx(fmaf(s[2 * cc], kScaleLog2, neg_m)),
+                                              ex2_approx(fmaf(s[2 * cc + 1], kScaleLog2, neg_m)));
+                    // the row sum of the BF16 weights the PV product uses
+                    lp[c & 3] += __bfloat162float(pb.x) + __bfloat162float(pb.y);
+                    pk[c] = *reinterpret_cast<const uint32_t *>(&pb);
+                }
+                // P (BF16 pairs) over the S buffer's first 64 columns
+                tmem_st16(tmem + lane_off + sb * 128u + static_cast<uint32_t>(col0 / 2 + 16 * h), pk);
             }
             l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
-            tmem_st32(tmem + lane_off + sb * 128u + wg * 32u, pk);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(p_full + 8 * sb);
         }
-        // epilogue: O / l -> BF16 (this half's 64 columns), and max |o|
+        // epilogue: O / l -> BF16 (this group's kCols columns), and max |o|
         lsum[wg * 128 + r] = l;
-        asm volatile("bar.sync 3, 256;" ::: "memory");
-        l += lsum[(1 - wg) * 128 + r];
+        asm volatile("bar.sync 3, %0;" ::"n"(32 * kSoftmaxWarps) : "memory");
+        l = 0.0f;
+#pragma unroll
+        for (int w2 = 0; w2 < kColGroups; ++w2) l += lsum[w2 * 128 + r];
         ok = __all_sync(0xFFFFFFFFu,
                         wait_bar(pv_done + 8 * ((nkv - 1) % kSBufs), ((nkv - 1) / kSBufs) & 1)) && ok;
         tc_fence_after();
@@ -323,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float omax = 0.0f;
         __nv_bfloat16 *orow = p.o + static_cast<int64_t>(row) * (p.H * kD) + h * kD + col0;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < kCols / 32; ++c) {
             uint32_t ov[32];
             tmem_ld32(tmem + lane_off + kOCol + col0 + c * 32u, ov);
             tmem_ld_wait();
@@ -344,9 +397,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (row >= p.M) omax = 0.0f;
         const uint32_t b = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(omax));
-        if (lane == 0) red[warp - 2] = __uint_as_float(b);
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-        if (warp == 2 && lane == 0) {
+        if (lane == 0) red[warp - kSoftWarp0] = __uint_as_float(b);
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * kSoftmaxWarps) : "memory");
+        if (warp == kSoftWarp0 && lane == 0) {
             float m = 0.0f;
             for (int i = 0; i < kSoftmaxWarps; ++i) m = fmaxf(m, red[i]);
             if (p.partial_slots > 0)
