@@ -588,27 +588,33 @@ def measure_layer(args, mq, dev, stream, flush, capture, replay_ms, pk):
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
 
-    def timed(fn, n):
-        fn()
-        torch.cuda.synchronize()
-        ts = []
-        for _ in range(n):
-            flush()
-            a, b = ev(), ev()
-            a.record(stream)
+    def timed_interleaved(fns, n):
+        """Median event time of each function, the functions taking turns
+        (each after an L2 flush) so that all of them see the same clock and
+        power state; this measurement follows seconds of dense GEMMs."""
+        for fn in fns:
             fn()
-            b.record(stream)
-            torch.cuda.synchronize()
-            ts.append(a.elapsed_time(b))
-        return statistics.median(ts)
+        torch.cuda.synchronize()
+        ts = [[] for _ in fns]
+        for _ in range(n):
+            for i, fn in enumerate(fns):
+                flush()
+                a, b = ev(), ev()
+                a.record(stream)
+                fn()
+                b.record(stream)
+                torch.cuda.synchronize()
+                ts[i].append(a.elapsed_time(b))
+        return [statistics.median(t) for t in ts]
 
     n = max(3, args.config_steps)
-    t_nv = timed(nvfp4_layer, n)
+    nvfp4_layer()
+    torch.cuda.synchronize()
     if mq.mq_check(stream) != 0:
         raise RuntimeError("device error in the layer")
-    t_attn = timed(attn, n)
-    t_sdpa = timed(sdpa, n)
-    t_bf = timed(bf16_layer, n)
+    t_nv, t_attn, t_sdpa, t_bf = timed_interleaved([nvfp4_layer, attn, sdpa, bf16_layer], n)
+    if mq.mq_check(stream) != 0:
+        raise RuntimeError("device error in the layer")
     attn_flops = 4.0 * Dh * H * M * (M + 1) / 2
     lin_flops = 2.0 * M * E * (Nqkv + E + 2 * I) + 2.0 * M * I * E
     r = {"workload": "llama3-8b layer (rmsnorm, qkv, causal gqa attention + kv cache, o, rmsnorm, "
@@ -624,7 +630,7 @@ def measure_layer(args, mq, dev, stream, flush, capture, replay_ms, pk):
          "attention_flops": attn_flops, "linear_flops": lin_flops,
          "note": "NVFP4 layer: this library's kernels only; BF16 layer: torch rms_norm, cuBLAS, "
                  "torch SDPA (flash/cuDNN) + cache copy; sdpa_ms includes the K/V cache copy; "
-                 "L2 flushed before each timed layer; medians of event-timed runs"}
+                 "L2 flushed before each timed layer; medians of event-timed runs, the four functions taking turns"}
     # decode step's attention block on the cache the prefill wrote: BF16 QKV
     # -> attention over 8192 + m positions -> BF16 O (device time, graph replays)
     R = 16
