@@ -1136,29 +1136,35 @@ def run_sharded(args, wl, world, rank):
 def profile_case(name: str):
     """Runs one small case a few times for a kernel capture (ncu -k ... -c 1):
     attention_prefill (4096 tokens, 8 query / 2 KV heads, head dim 128),
-    attention_decode (1 token over that cache), decode_nvfp4 (one token
-    through the Llama-3-8B QKV weight, W4A4)."""
+    attention_decode (1 token over a 32768-position cache, 32 query / 8 KV
+    heads), decode_nvfp4 (one token through the Llama-3-8B QKV weight, W4A4)."""
     from nvfp4_quantized_prefill_b200 import binding as mq
     mq.lib()
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     g = torch.Generator(device="cuda")
     g.manual_seed(9)
-    if name.startswith("attention"):
+    if name == "attention_prefill":
         M, H, Hkv, D = 4096, 8, 2, 128
-        qkv = torch.randn(M + 1, (H + 2 * Hkv) * D, device=dev, generator=g).to(torch.bfloat16)
+        qkv = torch.randn(M, (H + 2 * Hkv) * D, device=dev, generator=g).to(torch.bfloat16)
         kc = torch.zeros(Hkv, M + 8, D, dtype=torch.bfloat16, device=dev)
         vc = torch.zeros_like(kc)
         o = torch.empty(M, H * D, dtype=torch.bfloat16, device=dev)
         part = torch.empty(mq.MQ_AMAX_PARTIALS_MAX, dtype=torch.float32, device=dev)
         for _ in range(3):
-            mq.mq_attention_prefill_bf16(qkv[:M], M, H, Hkv, D, kc, vc, M + 8, o, part)
-        if name == "attention_decode":
-            ot = torch.empty(1, H * D, dtype=torch.bfloat16, device=dev)
-            nb = mq.mq_attention_decode_workspace_bytes(1, M, H, Hkv, D)
-            ws = torch.empty(nb, dtype=torch.uint8, device=dev)
-            for _ in range(3):
-                mq.mq_attention_decode_bf16(qkv[M:M + 1], 1, M, H, Hkv, D, kc, vc, M + 8, ot, ws, nb)
+            mq.mq_attention_prefill_bf16(qkv, M, H, Hkv, D, kc, vc, M + 8, o, part)
+    elif name == "attention_decode":
+        # one token over a 32768-position cache at the Llama-3-8B head counts
+        # (134 MB of K and V, above the L2)
+        S, H, Hkv, D = 32768, 32, 8, 128
+        kc = torch.randn(Hkv, S + 8, D, device=dev, generator=g).to(torch.bfloat16)
+        vc = torch.randn(Hkv, S + 8, D, device=dev, generator=g).to(torch.bfloat16)
+        qkv = torch.randn(1, (H + 2 * Hkv) * D, device=dev, generator=g).to(torch.bfloat16)
+        ot = torch.empty(1, H * D, dtype=torch.bfloat16, device=dev)
+        nb = mq.mq_attention_decode_workspace_bytes(1, S, H, Hkv, D)
+        ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            mq.mq_attention_decode_bf16(qkv, 1, S, H, Hkv, D, kc, vc, S + 8, ot, ws, nb)
     elif name == "decode_nvfp4":
         w = (torch.randn(6144, 4096, device=dev, generator=g) * 0.02).to(torch.bfloat16)
         W = mq.Weight(w)

@@ -736,6 +736,179 @@ __global__ void __launch_bounds__(kDecThreads) attention_decode_kernel(const Dec
             }
 }
 
+// Up to 8 query rows (one or two new tokens of a grouped head): each warp
+// keeps its own running maximum, sum and o over its 16 keys of every block
+// (S, the softmax and P.V need no cross-warp exchange: one block barrier per
+// 64 keys, for the double buffer), and the four warps' partials are merged
+// once at the end of the span.  Three K / V blocks per CTA: two loads stay in
+// flight while a block is computed.
+constexpr int kDecWarpPPitch = 24;    // BF16 per row of a warp's P transpose area
+constexpr int kDecWarpStages = 3;    // K / V blocks in flight or in use per CTA
+constexpr uint32_t kDecWarpSmem = 2 * kDecWarpStages * kDecTileBytes + 8 * kDecQPitch * 2 + 4 * 8 * kDecWarpPPitch * 2;
+
+__global__ void __launch_bounds__(kDecThreads) attention_decode_warp_kernel(const DecodeParams p) {
+    extern __shared__ __align__(128) uint8_t dsm[];
+    const uint32_t kv0 = smem_u32(dsm);                     // K[3], V[3]: 6 x 16 KB
+    __nv_bfloat16 *qs = reinterpret_cast<__nv_bfloat16 *>(dsm + 2 * kDecWarpStages * kDecTileBytes);   // [8][136]
+    __nv_bfloat16 *pw = qs + 8 * kDecQPitch;                                           // [4][8][24]
+    const int c = blockIdx.x, g = blockIdx.y, tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
+    const int group = p.H / p.Hkv;
+    const int n_keys = p.pos0 + p.m;
+    const int cols = (p.H + 2 * p.Hkv) * kD;
+    const __nv_bfloat16 *kbase = p.k_cache + static_cast<int64_t>(g) * p.S_max * kD;
+    const __nv_bfloat16 *vbase = p.v_cache + static_cast<int64_t>(g) * p.S_max * kD;
+    const int key_begin = c * p.span_blocks * kDecKeys;
+    const int nb = min(p.span_blocks, (n_keys - key_begin + kDecKeys - 1) / kDecKeys);
+    auto load_block = [&](int b) {
+        const int key0 = key_begin + b * kDecKeys;
+        const uint32_t kdst = kv0 + static_cast<uint32_t>(b % kDecWarpStages) * kDecTileBytes;
+        const uint32_t vdst = kdst + kDecWarpStages * kDecTileBytes;
+        for (int i = tid; i < kDecKeys * (kD / 8); i += kDecThreads) {
+            const int k = i >> 4, ch = i & 15;
+            const bool in = key0 + k < n_keys;
+            const int64_t off = static_cast<int64_t>(in ? key0 + k : key0) * kD + ch * 8;
+            cp_async16(kdst + dec_tile_off(k, ch), kbase + off, in ? 16u : 0u);
+            cp_async16(vdst + dec_tile_off(k, ch), vbase + off, in ? 16u : 0u);
+        }
+        cp_async_commit();
+    };
+    griddep_wait();            // the appended rows and the queries are in place
+    griddep_launch_dependents();
+    load_block(0);
+    if (nb > 1) load_block(1);
+    for (int i = tid; i < 8 * (kD / 2); i += kDecThreads) {
+        const int rr = i / (kD / 2), d2 = (i % (kD / 2)) * 2;
+        uint32_t v = 0;
+        if (rr < p.rows) {
+            const int hh = rr / p.m, t = rr % p.m;
+            v = *reinterpret_cast<const uint32_t *>(p.qkv + static_cast<int64_t>(t) * cols + (g * group + hh) * kD + d2);
+        }
+        *reinterpret_cast<uint32_t *>(qs + rr * kDecQPitch + d2) = v;
+    }
+    // this warp's running state for rows 2 tq, 2 tq + 1 (the C-fragment
+    // columns) and its O^T: dims 16 i + gq (+ 8), rows 2 tq (+ 1)
+    float m_w[2] = {-INFINITY, -INFINITY}, l_w[2] = {0.0f, 0.0f};
+    float acc[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[i][e] = 0.0f;
+    __nv_bfloat16 *pwt = pw + warp * 8 * kDecWarpPPitch;
+    for (int b = 0; b < nb; ++b) {
+        // block b landed (block b + 1 may still be in flight)
+        if (b + 1 < nb)
+            cp_async_wait<1>();
+        else
+            cp_async_wait<0>();
+        __syncthreads();           // ... for every thread's copies; every warp is done with block b - 1
+        if (b + 2 < nb) load_block(b + 2);   // into the buffer block b - 1 used
+        const int key0 = key_begin + b * kDecKeys;
+        const uint32_t kt = kv0 + static_cast<uint32_t>(b % kDecWarpStages) * kDecTileBytes;
+        const uint32_t vt = kt + kDecWarpStages * kDecTileBytes;
+        float sc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int s = 0; s < kD / 16; ++s) {
+            uint32_t a[4];
+            ldsm_x4(kt + dec_tile_off(16 * warp + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * s + (lane >> 4)), a);
+            const __nv_bfloat16 *qr = qs + gq * kDecQPitch + 16 * s + 2 * tq;
+            mma_bf16_16816(sc, a, *reinterpret_cast<const uint32_t *>(qr),
+                           *reinterpret_cast<const uint32_t *>(qr + 8));
+        }
+        float mx[2];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int row = 2 * tq + (e & 1);
+            const int pos = key0 + 16 * warp + gq + (e >> 1) * 8;
+            const bool ok = row < p.rows && pos < n_keys && pos <= p.pos0 + row % p.m;
+            sc[e] = ok ? sc[e] * kScaleLog2 : -INFINITY;
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float v = fmaxf(sc[h], sc[h + 2]);
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+            mx[h] = v;
+        }
+        float sum[2] = {0.0f, 0.0f}, alpha[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const float m_new = fmaxf(m_w[h], mx[h]);
+            alpha[h] = m_w[h] == -INFINITY ? 0.0f : exp2f(m_w[h] - m_new);
+            m_w[h] = m_new;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int h = e & 1;
+            const float w = m_w[h] == -INFINITY ? 0.0f : exp2f(sc[e] - m_w[h]);
+            const __nv_bfloat16 wb = __float2bfloat16_rn(w);
+            sum[h] += __bfloat162float(wb);
+            pwt[(2 * tq + h) * kDecWarpPPitch + gq + (e >> 1) * 8] = wb;
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float v = sum[h];
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+            l_w[h] = l_w[h] * alpha[h] + v;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            acc[i][0] *= alpha[0];
+            acc[i][1] *= alpha[1];
+            acc[i][2] *= alpha[0];
+            acc[i][3] *= alpha[1];
+        }
+        __syncwarp();              // this warp's P transpose is complete
+        const uint32_t b0 = *reinterpret_cast<const uint32_t *>(pwt + gq * kDecWarpPPitch + 2 * tq);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t *>(pwt + gq * kDecWarpPPitch + 2 * tq + 8);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            uint32_t a[4];
+            const int mi = lane >> 3;
+            ldsm_x4_trans(vt + dec_tile_off(16 * warp + (lane & 7) + (mi >> 1) * 8, 2 * i + (mi & 1)), a);
+            mma_bf16_16816(acc[i], a, b0, b1);
+        }
+        __syncwarp();              // P reads done before the next block's P is written
+    }
+    __syncthreads();               // the K / V buffers are free for the merge
+    // merge the four warps: per warp m and l of the 8 rows and O[8][128]
+    float *mw = reinterpret_cast<float *>(dsm);              // [4][8]
+    float *lw = mw + 32;                                      // [4][8]
+    float *ow = lw + 32;                                      // [4][8][128]
+    if (gq == 0) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            mw[warp * 8 + 2 * tq + h] = m_w[h];
+            lw[warp * 8 + 2 * tq + h] = l_w[h];
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            ow[(warp * 8 + 2 * tq + (e & 1)) * kD + 16 * i + gq + (e >> 1) * 8] = acc[i][e];
+    __syncthreads();
+    float *part = p.part + (static_cast<int64_t>(g) * p.n_chunks + c) * p.rows * (2 + kD);
+    for (int rr = 0; rr < p.rows; ++rr) {
+        float mm = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) mm = fmaxf(mm, mw[w * 8 + rr]);
+        float l = 0.0f, o = 0.0f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const float f = mw[w * 8 + rr] == -INFINITY ? 0.0f : exp2f(mw[w * 8 + rr] - mm);
+            l = fmaf(lw[w * 8 + rr], f, l);
+            o = fmaf(ow[(w * 8 + rr) * kD + tid], f, o);
+        }
+        if (tid == 0) {
+            part[rr * (2 + kD)] = mm;
+            part[rr * (2 + kD) + 1] = l;
+        }
+        part[rr * (2 + kD) + 2 + tid] = o;
+    }
+}
+
 template <int kNT>
 cudaError_t launch_decode_rows(const DecodeParams &p, cudaStream_t s) {
     constexpr uint32_t smem = dec_smem_bytes<kNT>();
@@ -824,8 +997,15 @@ cudaError_t launch_attention_decode(const void *qkv, int64_t m, int64_t pos0, in
     p.n_chunks = static_cast<int>((pos0 + m + span - 1) / span);
     cudaError_t e = launch_pdl(kv_append_kernel, dim3(p.m, p.Hkv), dim3(32), 0, s, p);
     if (e != cudaSuccess) return e;
-    e = p.rows <= 8 ? launch_decode_rows<1>(p, s)
-                    : (p.rows <= 32 ? launch_decode_rows<4>(p, s) : launch_decode_rows<kDecMaxRows / 8>(p, s));
+    if (p.rows <= 8) {
+        e = cudaFuncSetAttribute(attention_decode_warp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kDecWarpSmem);
+        if (e == cudaSuccess)
+            e = launch_pdl(attention_decode_warp_kernel, dim3(p.n_chunks, p.Hkv), dim3(kDecThreads),
+                           kDecWarpSmem, s, p);
+    } else {
+        e = p.rows <= 32 ? launch_decode_rows<4>(p, s) : launch_decode_rows<kDecMaxRows / 8>(p, s);
+    }
     if (e != cudaSuccess) return e;
     e = launch_pdl(attention_combine_kernel, dim3(p.rows, p.Hkv), dim3(kD * kCombineGroups), 0, s, p);
     return e != cudaSuccess ? e : cudaGetLastError();

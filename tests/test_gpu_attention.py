@@ -98,11 +98,15 @@ def test_prefill_attention_llama8b_shape_sampled_rows():
     assert mq.mq_check() == 0
 
 
-@pytest.mark.parametrize("S,m,H,Hkv", [(300, 1, 8, 2), (300, 4, 8, 2), (129, 8, 4, 1), (1, 16, 4, 4)])
+@pytest.mark.parametrize("S,m,H,Hkv", [(300, 1, 8, 2), (300, 4, 8, 2), (129, 8, 4, 1), (1, 16, 4, 4),
+                                       (1000, 9, 8, 2), (200, 16, 8, 2), (4032, 64, 2, 2), (6000, 3, 16, 4)])
 def test_decode_attention_after_prefill(S, m, H, Hkv):
     """Prefill S tokens into the cache, then decode m new tokens: each new
     token attends over the cached positions and the new ones up to itself --
-    the prefill rows S .. S+m-1 of the whole sequence."""
+    the prefill rows S .. S+m-1 of the whole sequence.  Query rows per KV
+    head (group x m) from 1 to 64 (one to eight 8-row tiles of the decode
+    kernel), caches ending inside a 64-key block and on its boundary
+    (4032 + 64 = 4096), and spans of several blocks (6000 positions)."""
     S_max = S + m + 5
     qkv_all = _qkv(S + m, H, Hkv, 7 * S + m)
     _, kc, vc, _, _ = _prefill(qkv_all[:S].cuda().contiguous(), S, H, Hkv, S_max)
