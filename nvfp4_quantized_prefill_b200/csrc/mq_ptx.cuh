@@ -174,24 +174,8 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
                  : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-                 : "memory");
-}
-
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
-}
-
-// TMA tile load into this CTA's shared memory whose completion is counted on
-// an mbarrier that may live in the peer CTA of the pair (shared::cluster address).
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void *tmap, int32_t x, int32_t y,
-                                                 uint32_t bar_cluster) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(bar_cluster)
-        : "memory");
 }
 
 // ---- tcgen05, CTA-pair forms (cta_group::2) ----------------------------------------
@@ -209,40 +193,6 @@ __device__ __forceinline__ void tmem_alloc_pair(uint32_t dst, uint32_t ncols) {
 __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                  : "memory");
-}
-
-// Arrive on the mbarrier at this shared offset in every CTA of `cta_mask`
-// once this thread's earlier tcgen05 operations have completed.
-__device__ __forceinline__ void tc_commit_pair_mc(uint32_t bar, uint16_t cta_mask) {
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-        " [%0], %1;" ::"r"(bar),
-        "h"(cta_mask)
-        : "memory");
-}
-
-// Same, to one local mbarrier.
-__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
-}
-
-__device__ __forceinline__ void tc_cp_sf_pair(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-                 : "memory");
-}
-
-// M = 256 across the pair (128 rows per CTA), K = 64, E2M1 x E2M1 with UE4M3 scales.
-__device__ __forceinline__ void tc_mma_nvf4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                                 uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
-                                                 uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16"
-        " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-        : "memory");
 }
 
 // ---- warp-issued forms -------------------------------------------------------------
@@ -476,61 +426,11 @@ __device__ __forceinline__ void tmem_st_wait() {
 
 // ---- tcgen05, single-CTA BF16 forms (kind::f16) -------------------------------------
 
-// D (TMEM, FP32) (+)= A * B, A and B BF16 from shared memory (descriptors),
-// M = 128, K = 16 per call.
-__device__ __forceinline__ void tc_mma_bf16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                               uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Same with A (M x K, BF16, one row per lane, two elements per 32-bit column)
-// read from tensor memory.
-__device__ __forceinline__ void tc_mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
-                                               uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Eight chained BF16 MMAs (K = 8 x 16) and a commit, from one issue block:
-// A and B from shared memory, K-major with 128-byte swizzle, the K steps 32
-// bytes apart inside a 64-element atom and `atom_bytes` apart across the two
-// atoms; the first MMA overwrites D when `accumulate` is 0.
-__device__ __forceinline__ void tc_mma8_bf16_ss_commit(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                                       uint32_t idesc, uint32_t accumulate,
-                                                       uint32_t bar) {
-    asm volatile(
-        "{\n\t.reg .pred p, t;\n\t"
-        ".reg .b64 a1, a2, a3, a4, a5, a6, a7, b1, b2, b3, b4, b5, b6, b7;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\tsetp.eq.b32 t, 0, 0;\n\t"
-        "add.s64 a1, %1, 2;\n\tadd.s64 a2, %1, 4;\n\tadd.s64 a3, %1, 6;\n\t"
-        "add.s64 a4, %1, 1024;\n\tadd.s64 a5, %1, 1026;\n\tadd.s64 a6, %1, 1028;\n\t"
-        "add.s64 a7, %1, 1030;\n\t"
-        "add.s64 b1, %2, 2;\n\tadd.s64 b2, %2, 4;\n\tadd.s64 b3, %2, 6;\n\t"
-        "add.s64 b4, %2, 1024;\n\tadd.s64 b5, %2, 1026;\n\tadd.s64 b6, %2, 1028;\n\t"
-        "add.s64 b7, %2, 1030;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, t;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], a2, b2, %3, t;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], a3, b3, %3, t;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], a4, b4, %3, t;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], a5, b5, %3, t;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], a6, b6, %3, t;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], a7, b7, %3, t;\n\t"
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%5];\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(bar)
-        : "memory");
-}
-
-// The same, with two commits (two barriers track the MMAs' completion).
+// D (TMEM, FP32) (+)= A * B over K = 128: eight chained BF16 MMAs (M = 128,
+// K = 16 each) with A and B K-major 128-byte-swizzled shared-memory operands
+// (descriptors advanced by 32 bytes per step within a 64-column half of the
+// 128-column tile, and by 16 KB to the tile's second half after four steps),
+// then two commits: each barrier arrives once the MMAs have completed.
 __device__ __forceinline__ void tc_mma8_bf16_ss_commit2(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                                         uint32_t idesc, uint32_t accumulate,
                                                         uint32_t bar0, uint32_t bar1) {
