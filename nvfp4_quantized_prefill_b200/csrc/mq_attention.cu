@@ -79,6 +79,29 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// a * b + c on two FP32 lanes at once (packed pairs: element 0 in the low word)
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+    return d;
+}
+__device__ __forceinline__ void unpack_f32x2(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+// acc + both BF16 halves of w, each widened exactly to FP32 by the mixed-type FMA
+__device__ __forceinline__ float add_bf16x2_f32(float acc, uint32_t w) {
+    asm("{\n\t.reg .b16 lo, hi, one;\n\tmov.b32 {lo, hi}, %1;\n\tmov.b16 one, 0x3F80;\n\t"
+        "fma.rn.f32.bf16 %0, lo, one, %0;\n\tfma.rn.f32.bf16 %0, hi, one, %0;\n\t}"
+        : "+f"(acc)
+        : "r"(w));
+    return acc;
+}
+
 // Bounded wait on an mbarrier phase (all lanes poll); false after the limit.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -338,7 +361,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             l *= f;
             m_run = m_new;
-            const float neg_m = -m_run;
+            // exponents two at a time (packed FMA), the weights rounded to
+            // BF16 pairs, and their row sum taken over the rounded values
+            const uint64_t sc2 = pack_f32x2(kScaleLog2, kScaleLog2);
+            const uint64_t nm2 = pack_f32x2(-m_run, -m_run);
             float lp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
             for (int h = 0; h < kCols / 32; ++h) {
@@ -346,12 +372,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int c = 0; c < 16; ++c) {
                     const int cc = 16 * h + c;
-                    const __nv_bfloat162 pb =
-                        __floats2bfloat162_rn(ex2_approx(fmaf(s[2 * cc], kScaleLog2, neg_m)),
-                                              ex2_approx(fmaf(s[2 * cc + 1], kScaleLog2, neg_m)));
-                    // the row sum of the BF16 weights the PV product uses
-                    lp[c & 3] += __bfloat162float(pb.x) + __bfloat162float(pb.y);
+                    float x0, x1;
+                    unpack_f32x2(ffma2(pack_f32x2(s[2 * cc], s[2 * cc + 1]), sc2, nm2), x0, x1);
+                    const __nv_bfloat162 pb = __floats2bfloat162_rn(ex2_approx(x0), ex2_approx(x1));
                     pk[c] = *reinterpret_cast<const uint32_t *>(&pb);
+                    lp[c & 3] = add_bf16x2_f32(lp[c & 3], pk[c]);
                 }
                 // P (BF16 pairs) over the S buffer's first 64 columns
                 tmem_st16(tmem + lane_off + sb * 128u + static_cast<uint32_t>(col0 / 2 + 16 * h), pk);
