@@ -79,6 +79,12 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // a * b + c on two FP32 lanes at once (packed pairs: element 0 in the low word)
 __device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
     uint64_t d;
@@ -308,14 +314,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < kCols; ++c)
                     if (col0 + c > r) s[c] = -INFINITY;
             }
+            // eight chains of three-input maxima
             float mp[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) mp[e] = -INFINITY;
+            for (int e = 0; e < 8; ++e) mp[e] = fmaxf(s[e], s[8 + e]);
 #pragma unroll
-            for (int c = 0; c < kCols; ++c) mp[c & 7] = fmaxf(mp[c & 7], s[c]);   // eight chains
+            for (int c = 16; c < kCols; c += 16)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) mp[e] = fmax3(mp[e], s[c + e], s[c + 8 + e]);
             // the scale is positive: the maximum of the scaled scores
-            float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) * kScaleLog2;
+            float mx = fmaxf(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], fmax3(mp[5], mp[6], mp[7]))) *
+                       kScaleLog2;
             xchg[(st * kColGroups + wg) * 128 + r] = mx;
             // the barrier's AND also carries "every softmax warp saw S": after
             // a timed-out wait all softmax warps leave the loop together (none
