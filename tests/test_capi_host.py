@@ -137,3 +137,44 @@ def test_amax_shape_bound_at_the_32_bit_edge(lib):
     rows = ((1 << 32) - 2) // 512  # largest M with M * 512 < 2^32 - 1
     assert L.mq_tensor_amax(16, rows, 4096, 4096, 20, ctypes.byref(n), None) == 3
     assert L.mq_tensor_amax(16, rows + 1, 4096, 4096, 20, ctypes.byref(n), None) == 2
+
+
+def _dec_ws_expected(m, pos0, H, Hkv):
+    """Workspace of the decode attention, written out from its definition:
+    (max, sum, 128 partial outputs) in FP32 per query row and span, the
+    spans being runs of 64-key blocks, as few blocks as keep spans x KV
+    heads within 256."""
+    n_keys = pos0 + m
+    blocks = -(-n_keys // 64)
+    span_blocks = max(1, -(-(blocks * Hkv) // 256))
+    spans = -(-n_keys // (64 * span_blocks))
+    return Hkv * spans * (H // Hkv * m) * (2 + 128) * 4
+
+
+@pytest.mark.parametrize("m,pos0,H,Hkv", [(1, 0, 1, 1), (1, 63, 8, 2), (1, 64, 8, 2), (8, 8192, 32, 8),
+                                          (1, 65535, 32, 8), (16, 200, 8, 2), (3, 6000, 16, 4)])
+def test_decode_attention_workspace_bytes(lib, m, pos0, H, Hkv):
+    assert binding.mq_attention_decode_workspace_bytes(m, pos0, H, Hkv, 128) == _dec_ws_expected(m, pos0, H, Hkv)
+
+
+def test_attention_entry_points_reject_bad_arguments_on_the_host(lib):
+    L = lib
+    n = ctypes.c_int()
+    ws = binding.mq_attention_decode_workspace_bytes
+    # invalid sizes: no workspace at all
+    assert ws(1, 8, 8, 2, 64) == 0 and ws(0, 8, 8, 2, 128) == 0 and ws(1, 8, 8, 3, 128) == 0
+    assert ws(1, -1, 8, 2, 128) == 0
+    # prefill: null pointers, one cache pointer without the other, shapes, alignment
+    assert L.mq_attention_prefill_bf16(None, 16, 4, 2, 128, None, None, 0, 16, 16, ctypes.byref(n), None) == 1
+    assert L.mq_attention_prefill_bf16(16, 16, 4, 2, 128, 16, None, 16, 16, 16, ctypes.byref(n), None) == 1
+    assert L.mq_attention_prefill_bf16(16, 16, 4, 2, 64, None, None, 0, 16, 16, ctypes.byref(n), None) == 2
+    assert L.mq_attention_prefill_bf16(16, 16, 4, 3, 128, None, None, 0, 16, 16, ctypes.byref(n), None) == 2
+    assert L.mq_attention_prefill_bf16(16, 16, 4, 2, 128, 16, 16, 8, 16, 16, ctypes.byref(n), None) == 2
+    assert L.mq_attention_prefill_bf16(24, 16, 4, 2, 128, None, None, 0, 16, 16, ctypes.byref(n), None) == 3
+    # decode: rows per KV head above 64, the cache too short, workspace too small, alignment
+    big = 1 << 30
+    assert L.mq_attention_decode_bf16(None, 1, 8, 8, 2, 128, 16, 16, 16, 16, 16, big, None) == 1
+    assert L.mq_attention_decode_bf16(16, 17, 8, 8, 2, 128, 16, 16, 64, 16, 16, big, None) == 2
+    assert L.mq_attention_decode_bf16(16, 1, 8, 8, 2, 128, 16, 16, 8, 16, 16, big, None) == 2
+    assert L.mq_attention_decode_bf16(16, 1, 8, 8, 2, 128, 16, 16, 16, 16, 16, 16, None) == 1
+    assert L.mq_attention_decode_bf16(24, 1, 8, 8, 2, 128, 16, 16, 16, 16, 16, big, None) == 3
