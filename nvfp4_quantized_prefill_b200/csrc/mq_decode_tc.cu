@@ -249,11 +249,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t sSB = sSA + kSfBytes;
                 const uint32_t tsa = tmem + kSfCol + static_cast<uint32_t>(stage) * kSfColsPerStage;
                 const uint32_t tsb = tsa + 16u;
-                for (int kb = 0; kb < natoms; ++kb) {
-                    tc_cp_sf(tsa + 4u * kb, sdesc_sf_tile(sSA + 512u * kb));
-                    tc_cp_sf(tsb + 4u * kb, sdesc_sf_tile(sSB + 512u * kb));
+                if (natoms == 4) {
+                    tc_cp8_sf_commit(tsa, tsb, sdesc_sf_tile(sSA), sdesc_sf_tile(sSB), sff0 + 8u * stage);
+                } else {
+                    for (int kb = 0; kb < natoms; ++kb) {
+                        tc_cp_sf(tsa + 4u * kb, sdesc_sf_tile(sSA + 512u * kb));
+                        tc_cp_sf(tsb + 4u * kb, sdesc_sf_tile(sSB + 512u * kb));
+                    }
+                    tc_commit(sff0 + 8u * stage);
                 }
-                tc_commit(sff0 + 8u * stage);
                 if (++stage == kStages) {
                     stage = 0;
                     phase ^= 1u;
@@ -292,13 +296,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t sB = sA + kABytes;
                     const uint32_t tsa = tmem + kSfCol + static_cast<uint32_t>(stage) * kSfColsPerStage;
                     const uint32_t tsb = tsa + 16u;
-                    for (int kb = 0; kb < natoms; ++kb) {
-                        tc_mma_nvf4(dacc, sdesc_kmajor_sw128(sA + 32u * kb),
-                                    sdesc_kmajor_sw128(sB + 32u * kb), idesc, tsa + 4u * kb,
-                                    tsb + 4u * kb, accumulate);
+                    if (natoms == 4) {   // the stage's MMAs and the commit that frees it
+                        tc_mma4_nvf4_commit(dacc, sdesc_kmajor_sw128(sA), sdesc_kmajor_sw128(sB), idesc, tsa, tsb,
+                                            accumulate, empty0 + 8u * stage);
                         accumulate = 1;
+                    } else {
+                        for (int kb = 0; kb < natoms; ++kb) {
+                            tc_mma_nvf4(dacc, sdesc_kmajor_sw128(sA + 32u * kb),
+                                        sdesc_kmajor_sw128(sB + 32u * kb), idesc, tsa + 4u * kb,
+                                        tsb + 4u * kb, accumulate);
+                            accumulate = 1;
+                        }
+                        tc_commit(empty0 + 8u * stage);   // frees the stage
                     }
-                    tc_commit(empty0 + 8u * stage);   // frees the stage
                     if (++stage == kStages) {
                         stage = 0;
                         phase ^= 1u;
