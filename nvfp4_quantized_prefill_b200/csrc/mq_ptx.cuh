@@ -374,56 +374,6 @@ __device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uin
         : "memory");
 }
 
-// A whole 256-wide K stage from one thread in one issue block: four such MMAs
-// (K = 64 each: descriptors 32 bytes = 2 units apart, scale columns 4 apart),
-// the first accumulating only if `accumulate`, then a commit to `bar`.
-__device__ __forceinline__ void tc_mma4_nvf4_commit(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                                    uint32_t idesc, uint32_t sfa_tmem,
-                                                    uint32_t sfb_tmem, uint32_t accumulate,
-                                                    uint32_t bar) {
-    asm volatile(
-        "{\n\t.reg .pred p, t;\n\t"
-        ".reg .b64 a1, a2, a3, b1, b2, b3;\n\t"
-        ".reg .b32 sa1, sa2, sa3, sb1, sb2, sb3;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\tsetp.eq.b32 t, 0, 0;\n\t"
-        "add.s64 a1, %1, 2;\n\tadd.s64 a2, %1, 4;\n\tadd.s64 a3, %1, 6;\n\t"
-        "add.s64 b1, %2, 2;\n\tadd.s64 b2, %2, 4;\n\tadd.s64 b3, %2, 6;\n\t"
-        "add.u32 sa1, %5, 4;\n\tadd.u32 sa2, %5, 8;\n\tadd.u32 sa3, %5, 12;\n\t"
-        "add.u32 sb1, %6, 4;\n\tadd.u32 sb2, %6, 8;\n\tadd.u32 sb3, %6, 12;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], a1, b1, %3, [sa1], [sb1], t;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], a2, b2, %3, [sa2], [sb2], t;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], a3, b3, %3, [sa3], [sb3], t;\n\t"
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%7];\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem), "r"(bar)
-        : "memory");
-}
-
-// The four A and four B scale tiles of a 256-wide K stage (512-byte tiles,
-// 32 descriptor units apart) into TMEM columns 4 apart, then a commit to
-// `bar`, from one thread in one issue block.
-__device__ __forceinline__ void tc_cp8_sf_commit(uint32_t tsa, uint32_t tsb, uint64_t da, uint64_t db,
-                                                 uint32_t bar) {
-    asm volatile(
-        "{\n\t.reg .b64 a1, a2, a3, b1, b2, b3;\n\t"
-        ".reg .b32 ta1, ta2, ta3, tb1, tb2, tb3;\n\t"
-        "add.s64 a1, %2, 32;\n\tadd.s64 a2, %2, 64;\n\tadd.s64 a3, %2, 96;\n\t"
-        "add.s64 b1, %3, 32;\n\tadd.s64 b2, %3, 64;\n\tadd.s64 b3, %3, 96;\n\t"
-        "add.u32 ta1, %0, 4;\n\tadd.u32 ta2, %0, 8;\n\tadd.u32 ta3, %0, 12;\n\t"
-        "add.u32 tb1, %1, 4;\n\tadd.u32 tb2, %1, 8;\n\tadd.u32 tb3, %1, 12;\n\t"
-        "tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %2;\n\t"
-        "tcgen05.cp.cta_group::1.32x128b.warpx4 [%1], %3;\n\t"
-        "tcgen05.cp.cta_group::1.32x128b.warpx4 [ta1], a1;\n\t"
-        "tcgen05.cp.cta_group::1.32x128b.warpx4 [tb1], b1;\n\t"
-        "tcgen05.cp.cta_group::1.32x128b.warpx4 [ta2], a2;\n\t"
-        "tcgen05.cp.cta_group::1.32x128b.warpx4 [tb2], b2;\n\t"
-        "tcgen05.cp.cta_group::1.32x128b.warpx4 [ta3], a3;\n\t"
-        "tcgen05.cp.cta_group::1.32x128b.warpx4 [tb3], b3;\n\t"
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%4];\n\t}" ::"r"(tsa),
-        "r"(tsb), "l"(da), "l"(db), "r"(bar)
-        : "memory");
-}
-
 // 32 lanes x 32 consecutive 32-bit columns: thread t of the warp receives lane
 // (warp's lane group base + t), columns [col, col+32).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
