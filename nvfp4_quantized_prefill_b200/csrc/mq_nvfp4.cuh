@@ -56,11 +56,12 @@ __device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
 }
 
 // Eight BF16 values (two per word, element 2j in the low half of word j)
-// times f, each product rounded to FP32 (packed f32x2 multiplies) and then to
-// E2M1 (round-to-nearest-even, saturating at 6, the sign of x kept even when
-// the code is zero); returns the four code bytes, element 2j in the low
-// nibble of byte j.  kToMemory: the bytes are packed with one vector mov of
-// the four 8-bit results (the quantizer, whose codes go to memory).
+// times f, each product rounded to FP32 and then to E2M1 (round-to-nearest-
+// even, saturating at 6, the sign of x kept even when the code is zero);
+// returns the four code bytes, element 2j in the low nibble of byte j.  The
+// products are scalar FP32 multiplies: the packed f32x2 form measured ~12%
+// slower in the quantizer.  kToMemory: the bytes are packed with one vector
+// mov of the four 8-bit results (the quantizer, whose codes go to memory).
 // Otherwise they are widened and combined with integer arithmetic: a packed
 // word that was unpacked again into 8-bit registers in the same kernel,
 // without passing through memory, was observed to lose its top byte.
@@ -71,19 +72,15 @@ __device__ __forceinline__ uint32_t e2m1x8(uint32_t w0, uint32_t w1, uint32_t w2
     if (kToMemory) {
         asm("{\n\t"
             ".reg .b8 c0, c1, c2, c3;\n\t"
-            ".reg .b64 f2, x0, x1, x2, x3;\n\t"
             ".reg .b32 l0, h0, l1, h1, l2, h2, l3, h3;\n\t"
-            "mov.b64 f2, {%5, %5};\n\t"
             "shl.b32 l0, %1, 16;\n\tand.b32 h0, %1, 0xFFFF0000;\n\t"
             "shl.b32 l1, %2, 16;\n\tand.b32 h1, %2, 0xFFFF0000;\n\t"
             "shl.b32 l2, %3, 16;\n\tand.b32 h2, %3, 0xFFFF0000;\n\t"
             "shl.b32 l3, %4, 16;\n\tand.b32 h3, %4, 0xFFFF0000;\n\t"
-            "mov.b64 x0, {l0, h0};\n\tmov.b64 x1, {l1, h1};\n\t"
-            "mov.b64 x2, {l2, h2};\n\tmov.b64 x3, {l3, h3};\n\t"
-            "mul.rn.f32x2 x0, x0, f2;\n\tmul.rn.f32x2 x1, x1, f2;\n\t"
-            "mul.rn.f32x2 x2, x2, f2;\n\tmul.rn.f32x2 x3, x3, f2;\n\t"
-            "mov.b64 {l0, h0}, x0;\n\tmov.b64 {l1, h1}, x1;\n\t"
-            "mov.b64 {l2, h2}, x2;\n\tmov.b64 {l3, h3}, x3;\n\t"
+            "mul.rn.f32 l0, l0, %5;\n\tmul.rn.f32 h0, h0, %5;\n\t"
+            "mul.rn.f32 l1, l1, %5;\n\tmul.rn.f32 h1, h1, %5;\n\t"
+            "mul.rn.f32 l2, l2, %5;\n\tmul.rn.f32 h2, h2, %5;\n\t"
+            "mul.rn.f32 l3, l3, %5;\n\tmul.rn.f32 h3, h3, %5;\n\t"
             "cvt.rn.satfinite.e2m1x2.f32 c0, h0, l0;\n\t"
             "cvt.rn.satfinite.e2m1x2.f32 c1, h1, l1;\n\t"
             "cvt.rn.satfinite.e2m1x2.f32 c2, h2, l2;\n\t"
@@ -95,19 +92,15 @@ __device__ __forceinline__ uint32_t e2m1x8(uint32_t w0, uint32_t w1, uint32_t w2
     } else {
         asm("{\n\t"
             ".reg .b8 c0, c1, c2, c3;\n\t"
-            ".reg .b64 f2, x0, x1, x2, x3;\n\t"
             ".reg .b32 l0, h0, l1, h1, l2, h2, l3, h3;\n\t"
-            "mov.b64 f2, {%5, %5};\n\t"
             "shl.b32 l0, %1, 16;\n\tand.b32 h0, %1, 0xFFFF0000;\n\t"
             "shl.b32 l1, %2, 16;\n\tand.b32 h1, %2, 0xFFFF0000;\n\t"
             "shl.b32 l2, %3, 16;\n\tand.b32 h2, %3, 0xFFFF0000;\n\t"
             "shl.b32 l3, %4, 16;\n\tand.b32 h3, %4, 0xFFFF0000;\n\t"
-            "mov.b64 x0, {l0, h0};\n\tmov.b64 x1, {l1, h1};\n\t"
-            "mov.b64 x2, {l2, h2};\n\tmov.b64 x3, {l3, h3};\n\t"
-            "mul.rn.f32x2 x0, x0, f2;\n\tmul.rn.f32x2 x1, x1, f2;\n\t"
-            "mul.rn.f32x2 x2, x2, f2;\n\tmul.rn.f32x2 x3, x3, f2;\n\t"
-            "mov.b64 {l0, h0}, x0;\n\tmov.b64 {l1, h1}, x1;\n\t"
-            "mov.b64 {l2, h2}, x2;\n\tmov.b64 {l3, h3}, x3;\n\t"
+            "mul.rn.f32 l0, l0, %5;\n\tmul.rn.f32 h0, h0, %5;\n\t"
+            "mul.rn.f32 l1, l1, %5;\n\tmul.rn.f32 h1, h1, %5;\n\t"
+            "mul.rn.f32 l2, l2, %5;\n\tmul.rn.f32 h2, h2, %5;\n\t"
+            "mul.rn.f32 l3, l3, %5;\n\tmul.rn.f32 h3, h3, %5;\n\t"
             "cvt.rn.satfinite.e2m1x2.f32 c0, h0, l0;\n\t"
             "cvt.rn.satfinite.e2m1x2.f32 c1, h1, l1;\n\t"
             "cvt.rn.satfinite.e2m1x2.f32 c2, h2, l2;\n\t"
