@@ -86,6 +86,19 @@ def recorded_traffic(workload_key: str):
     return sum(per.values()) / len(per), sorted(per)
 
 
+def recorded_tensor_pipe(workload_key: str):
+    """ncu's tensor-pipe activity (% of elapsed cycles) per GEMM launch from
+    the same committed capture as the traffic, only if it was taken on the
+    GEMM source as it is now; None otherwise."""
+    try:
+        d = json.load(open(COUNTERS))
+    except Exception:
+        return None
+    if d.get("gemm_source_hash") != gemm_source_hash():
+        return None
+    return d.get("gemm_tensor_pipe_active_pct", {}).get(workload_key)
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples during the timed region."""
 
@@ -1037,6 +1050,9 @@ def run_gpu(args, wl, world, rank):
             "frac": round(achieved / fp4_peak, 4),
             "traffic": traffic,
             "traffic_launches": traffic_launches,
+            # read beside frac: frac is against 4x the measured BF16 burst,
+            # this is the tensor pipe's own busy fraction under ncu
+            "tensor_pipe_active_pct_ncu": recorded_tensor_pipe(args.workload),
             "launches_per_step": n_gemm,
         },
         "e2e": e2e,

@@ -58,6 +58,11 @@ def test_recorded_traffic_only_for_the_current_gemm_source(tmp_path, monkeypatch
     p.write_text(json.dumps(stale))
     monkeypatch.setattr(bench, "COUNTERS", str(p))
     assert bench.recorded_traffic("llama3_8b_qkv_o") == (None, None)
+    assert bench.recorded_tensor_pipe("llama3_8b_qkv_o") is None
     # nor a workload without a capture
     monkeypatch.setattr(bench, "COUNTERS", orig)
     assert bench.recorded_traffic("no_such_workload") == (None, None)
+    assert bench.recorded_tensor_pipe("no_such_workload") is None
+    if d["gemm_source_hash"] == bench.gemm_source_hash():
+        pipe = bench.recorded_tensor_pipe("llama3_8b_qkv_o")
+        assert set(pipe) == set(per) and all(0.0 < v <= 100.0 for v in pipe.values())
