@@ -14,15 +14,17 @@
 //
 // Prefill kernel: one CTA per (128-query tile, query head), heaviest tiles
 // first.  Warp 0 loads Q once and K / V tiles (TMA, 128-byte swizzle) into a
-// 2-stage ring; warp 1 issues S = Q K^T (kind::f16, M = 128, N = 128, K = 16
-// per instruction) into one of two 128-column FP32 buffers in tensor memory,
-// and O += P V with P read from tensor memory; warps 2-9 (two threads per
-// query row, 64 columns each) take the row maximum, raise the running maximum only when it grows
-// by more than 2^8 (then O is rescaled in place; otherwise the stale maximum
-// keeps every weight below 2^8 and the final division by the same-based sum is
-// exact), write P as BF16 over the S buffer, and finally divide O by the row
-// sum, store it and keep max |o| for the O projection's quantizer.  The first
-// query head of each KV group writes its diagonal K / V tile to the cache.
+// 2-stage ring, K and V released separately; warp 1 issues S = Q K^T
+// (kind::f16, M = 128, N = 128, K = 16 per instruction) into one of three
+// 128-column FP32 buffers in tensor memory; warp 2 issues O += P V with P
+// read from tensor memory; warps 3-6 (one thread per query row, all 128
+// columns of its S row: no exchange between threads) take the row maximum,
+// raise the running maximum only when it grows by more than 2^8 (then O is
+// rescaled in place; otherwise the stale maximum keeps every weight below 2^8
+// and the final division by the same-based sum is exact), write P as BF16
+// over the S buffer, and finally divide O by the row sum, store it and keep
+// max |o| for the O projection's quantizer.  The first query head of each KV
+// group writes its diagonal K / V tile to the cache.
 #include <cuda_bf16.h>
 
 #include <cstring>
@@ -44,9 +46,12 @@ constexpr uint32_t kKOff = kTileBytes;                       // K stages
 constexpr uint32_t kVOff = kKOff + kStages * kTileBytes;     // V stages
 constexpr uint32_t kBarOff = kVOff + kStages * kTileBytes;
 #ifndef MQ_ATT_COL_GROUPS
-#define MQ_ATT_COL_GROUPS 2
+#define MQ_ATT_COL_GROUPS 1
 #endif
-constexpr int kColGroups = MQ_ATT_COL_GROUPS;   // softmax warpgroups, each a column range of every row
+// softmax warpgroups, each a column range of every row: one (a thread owns
+// its whole S row) measured 4% faster on the 8B shape than two (half rows,
+// row maxima exchanged through shared memory and a named barrier per tile)
+constexpr int kColGroups = MQ_ATT_COL_GROUPS;
 constexpr int kCols = 128 / kColGroups;          // S columns per softmax thread
 constexpr uint32_t kXchgOff = kBarOff + 256;     // row maxima, 2 tiles x kColGroups x 128
 constexpr uint32_t kLsumOff = kXchgOff + 2 * kColGroups * 128 * 4;   // row sums, kColGroups x 128
@@ -284,10 +289,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else {
         // ---------------------------------------------------------- softmax
-        // warpgroup wg holds columns [kCols wg, kCols wg + kCols) of every row;
-        // the kColGroups threads of a row agree on the row maximum through
-        // shared memory (one named barrier a tile, double-buffered by tile
-        // parity) and keep their own share of the row sum
+        // warpgroup wg holds columns [kCols wg, kCols wg + kCols) of every row
+        // (all of them with one group); with several groups the threads of a
+        // row agree on the row maximum through shared memory (one named
+        // barrier a tile, double-buffered by tile parity) and keep their own
+        // share of the row sum
         const int wg = (warp - kSoftWarp0) >> 2;
         const int quarter = warp & 3;             // TMEM lane group of this warp
         const int r = quarter * 32 + lane;        // query row in the tile
@@ -325,27 +331,36 @@ __global__ void __launch_bounds__(kThreads, 1)
             // the scale is positive: the maximum of the scaled scores
             float mx = fmaxf(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], fmax3(mp[5], mp[6], mp[7]))) *
                        kScaleLog2;
-            xchg[(st * kColGroups + wg) * 128 + r] = mx;
-            // the barrier's AND also carries "every softmax warp saw S": after
-            // a timed-out wait all softmax warps leave the loop together (none
-            // may be left waiting here for the others); it also orders every
-            // thread's S loads before any thread's P stores over the buffer
-            uint32_t all_ok;
-            asm volatile(
-                "{\n\t.reg .pred p, q;\n\t"
-                "setp.ne.u32 p, %1, 0;\n\t"
-                "bar.red.and.pred q, 2, %2, p;\n\t"
-                "selp.u32 %0, 1, 0, q;\n\t}"
-                : "=r"(all_ok)
-                : "r"(ok ? 1u : 0u), "n"(32 * kSoftmaxWarps)
-                : "memory");
-            if (!all_ok) {
-                ok = false;
-                break;
-            }
+            if constexpr (kColGroups > 1) {
+                xchg[(st * kColGroups + wg) * 128 + r] = mx;
+                // the barrier's AND also carries "every softmax warp saw S":
+                // after a timed-out wait all softmax warps leave the loop
+                // together (none may be left waiting here for the others); it
+                // also orders every thread's S loads before any thread's P
+                // stores over the buffer
+                uint32_t all_ok;
+                asm volatile(
+                    "{\n\t.reg .pred p, q;\n\t"
+                    "setp.ne.u32 p, %1, 0;\n\t"
+                    "bar.red.and.pred q, 2, %2, p;\n\t"
+                    "selp.u32 %0, 1, 0, q;\n\t}"
+                    : "=r"(all_ok)
+                    : "r"(ok ? 1u : 0u), "n"(32 * kSoftmaxWarps)
+                    : "memory");
+                if (!all_ok) {
+                    ok = false;
+                    break;
+                }
 #pragma unroll
-            for (int w2 = 0; w2 < kColGroups; ++w2)
-                if (w2 != wg) mx = fmaxf(mx, xchg[(st * kColGroups + w2) * 128 + r]);
+                for (int w2 = 0; w2 < kColGroups; ++w2)
+                    if (w2 != wg) mx = fmaxf(mx, xchg[(st * kColGroups + w2) * 128 + r]);
+            } else {
+                // one thread per row: the row maximum is the thread's own, and
+                // a warp overwrites S only in its own TMEM lanes; a timed-out
+                // warp leaves on its own (the others run into their own
+                // bounded waits and meet it at the epilogue's barriers)
+                if (!ok) break;
+            }
             // raise the running maximum only for a growth beyond 2^8 (or at
             // the first tile); O then needs the factor 2^(m_old - m_new)
             const bool need = mx > m_run + kRescaleThreshold;
@@ -397,11 +412,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(p_full + 8 * sb);
         }
         // epilogue: O / l -> BF16 (this group's kCols columns), and max |o|
-        lsum[wg * 128 + r] = l;
-        asm volatile("bar.sync 3, %0;" ::"n"(32 * kSoftmaxWarps) : "memory");
-        l = 0.0f;
+        if constexpr (kColGroups > 1) {
+            lsum[wg * 128 + r] = l;
+            asm volatile("bar.sync 3, %0;" ::"n"(32 * kSoftmaxWarps) : "memory");
+            l = 0.0f;
 #pragma unroll
-        for (int w2 = 0; w2 < kColGroups; ++w2) l += lsum[w2 * 128 + r];
+            for (int w2 = 0; w2 < kColGroups; ++w2) l += lsum[w2 * 128 + r];
+        }
         ok = __all_sync(0xFFFFFFFFu,
                         wait_bar(pv_done + 8 * ((nkv - 1) % kSBufs), ((nkv - 1) / kSBufs) & 1)) && ok;
         tc_fence_after();
