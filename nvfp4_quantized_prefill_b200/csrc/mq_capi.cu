@@ -678,8 +678,9 @@ mq_status mq_decode_linear_nvfp4(const mq_weight *w, const void *x_bf16, int64_t
     if (mq::decode_nvf4_gemv_fits(M, w->K) && w->N * w->K <= (int64_t(1) << 25))
         return cuda_status(mq::launch_decode_nvf4_gemv(w->codes, w->sf, w->s_enc, w->N, w->K, x_bf16,
                                                        M, y_bf16, d->num_sms, stream));
+    const bool tc_fits = M <= mq::kDecodeTcTokens &&
+                         mq::decode_tc_token_bytes(M, w->N, w->K, d->num_sms) <= mq::kDecodeTcTokenSmem;
     const size_t tok_bytes = static_cast<size_t>(M) * static_cast<size_t>(w->K) * 9u / 16u;
-    const bool tc_fits = M <= mq::kDecodeTcTokens && tok_bytes + 15u <= mq::kDecodeTcTokenSmem;
     // the tensor-core kernel (quantizes the tokens itself, one pass over the
     // weight) for up to 4 tokens and for 9 to 16; for 5 to 8 only on weights
     // past 2^25 elements with M K <= 32768: there its stream beats the FP16

@@ -12,8 +12,9 @@
 //
 // The op streams the NVFP4 weight once (0.5625 byte per parameter); the
 // tensor core does the E2M1 decoding and the block scaling that an FP16 MMA
-// path spends most of its instructions on.  The tokens' NVFP4 form must fit
-// in shared memory (M K 9 / 16 <= kDecodeTcTokenSmem).  The weight is the
+// path spends most of its instructions on.  Each CTA quantizes the tokens
+// only over the K stages its units cover, and that NVFP4 form must fit in
+// shared memory (M x stages x 144 bytes <= kDecodeTcTokenSmem).  The weight is the
 // MMA's A operand (M = 128 weight rows) and the tokens its B operand (N = 16;
 // token rows past M stay zero), K = 64 per instruction with one UE4M3 scale
 // per 16 K.  Work unit: one 128-row weight tile x one 256-wide K stage; the
@@ -21,8 +22,9 @@
 // per CTA (one CTA per SM), so every SM streams the same bytes.  Each CTA's
 // few stages are short next to its fixed path (set-up, the first TMA round
 // trip, the token quantization, the accumulator hand-off and the cross-CTA
-// reduction), so the library uses it for up to 4 tokens and for 9 to 16; for
-// 5 to 8 the FP16-MMA kernel is faster.
+// reduction), so the library uses it for up to 4 tokens, for 9 to 16, and
+// for 5 to 8 on weights past 2^25 elements; for 5 to 8 tokens on smaller
+// weights the FP16-MMA kernel is faster.
 //
 // CTA roles (9 warps):
 //   warp 0     TMA producer: weight codes [128 x 128 B] (128-byte swizzle)
@@ -30,9 +32,9 @@
 //              8-stage ring.  The weight is constant for the call, so this
 //              warp starts before the wait for the preceding kernel.
 //   warps 2-5, 7-8  first, together: max |X| over all tokens (every CTA
-//              computes it), the scale table, and all of X quantized into
-//              shared memory (codes [M][K/2], scales [M][K/16]), while the
-//              weight streams in.
+//              computes it), the scale table, and X quantized into shared
+//              memory over the K stages of this CTA's units (codes, then
+//              scales, stage-major per token row), while the weight streams in.
 //   warps 7-8  then per stage: the token codes copied into the swizzled image
 //              the MMA reads and the token scales into their 512-byte tiles.
 //   warp 6     scale copier: copies a stage's scale tiles into tensor memory
@@ -68,7 +70,7 @@ constexpr uint32_t kStageBytes = kABytes + kBBytes + 2 * kSfBytes;   // 22528
 constexpr uint32_t kBarBytes = 512;
 constexpr uint32_t kTabBytes = 128 * 4 + 64;      // scale table + reduction scratch
 constexpr uint32_t kTokOff = kStages * kStageBytes + kBarBytes + kTabBytes;   // quantized tokens
-constexpr uint32_t kSmemFixed = kTokOff + 1024;   // + the tokens' M K 9/16 bytes
+constexpr uint32_t kSmemFixed = kTokOff + 1024;   // + the tokens' bytes (decode_tc_token_bytes)
 constexpr uint32_t kSmemMax = kSmemFixed + static_cast<uint32_t>(kDecodeTcTokenSmem);
 constexpr int kProducer = 0, kMma = 1, kEpi0 = 2, kCopier = 6, kQuant0 = 7;
 constexpr int kThreads = 9 * 32;
@@ -211,7 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int *last_flag = reinterpret_cast<volatile int *>(tmem_slot + 2);
     float *ftab = reinterpret_cast<float *>(smem + kStages * kStageBytes + kBarBytes);
     float *red = ftab + 128;   // 6 floats
-    uint8_t *xs = smem + kTokOff;   // codes [M][K/2], then scales [M][K/16]
+    uint8_t *xs = smem + kTokOff;   // this CTA's K stages of the tokens: codes, then scales
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -409,30 +411,73 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float s_enc = nvfp4_tensor_scale(amax);
         nvfp4_scale_table(s_enc, ftab, static_cast<uint32_t>(j), kPrologueThreads);
         named_bar_sync(kBarTok, kPrologueThreads);   // table complete
+        // Only the K stages this CTA's units cover are quantized (all of them
+        // once the range spans a whole tile), into a compact buffer: stage ks
+        // at slot so = (ks - ks0) mod kst, token row m holding n_st stages.
+        // Entry i = (m n_st + so) 16 + bb is 16-block bb of that stage:
+        // codes at 8 i, scale byte at xs_sf + i.
         const uint32_t kb16 = static_cast<uint32_t>(p.K / 16);   // 16-blocks per token row
-        const uint32_t nblk = static_cast<uint32_t>(p.M) * kb16;
-        uint8_t *xs_sf = xs + static_cast<uint32_t>(p.M) * static_cast<uint32_t>(p.K / 2);
-        for (uint32_t i0 = j; i0 < nblk; i0 += 4u * kPrologueThreads) {
-            uint4 v[4][2];
+        const int64_t nu = u1 - u0;
+        const int n_st = nu >= p.kst ? p.kst : static_cast<int>(nu);
+        const int ks0 = nu >= p.kst ? 0 : static_cast<int>(u0 % p.kst);
+        const uint32_t per_row = static_cast<uint32_t>(n_st) * 16u;   // blocks per token row
+        const uint32_t nblk = static_cast<uint32_t>(p.M) * per_row;
+        uint8_t *xs_sf = xs + 8u * nblk;
+        // every stage, and whole stages of 16 blocks: entry i is block i of X
+        // (the loop without the compact index arithmetic, which measured
+        // ~0.6 us slower on the 8B gate/up weight at one token)
+        const bool whole = n_st == p.kst && per_row == kb16;
+        auto quant_entry = [&](uint32_t i, const uint4 &a0, const uint4 &a1) {
+            const uint32_t w8[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            uint32_t lo, hi, sb;
+            quantize_block16<true>(w8, s_enc, ftab, lo, hi, sb);
+            *reinterpret_cast<uint2 *>(xs + 8u * i) = make_uint2(lo, hi);
+            xs_sf[i] = static_cast<uint8_t>(sb);
+        };
+        if (whole) {
+            for (uint32_t i0 = j; i0 < nblk; i0 += 4u * kPrologueThreads) {
+                uint4 v[4][2];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint32_t i = i0 + k * kPrologueThreads;   // block i: row i / kb16
-                v[k][0] = v[k][1] = make_uint4(0, 0, 0, 0);
-                if (i < nblk) {
-                    v[k][0] = __ldg(p.x + 2u * i);
-                    v[k][1] = __ldg(p.x + 2u * i + 1u);
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t i = i0 + k * kPrologueThreads;
+                    v[k][0] = v[k][1] = make_uint4(0, 0, 0, 0);
+                    if (i < nblk) {
+                        v[k][0] = __ldg(p.x + 2u * i);
+                        v[k][1] = __ldg(p.x + 2u * i + 1u);
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t i = i0 + k * kPrologueThreads;
+                    if (i >= nblk) break;
+                    quant_entry(i, v[k][0], v[k][1]);
                 }
             }
+        } else {
+            for (uint32_t i0 = j; i0 < nblk; i0 += 4u * kPrologueThreads) {
+                uint4 v[4][2];
+                bool valid[4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint32_t i = i0 + k * kPrologueThreads;
-                if (i >= nblk) break;
-                const uint32_t w8[8] = {v[k][0].x, v[k][0].y, v[k][0].z, v[k][0].w,
-                                        v[k][1].x, v[k][1].y, v[k][1].z, v[k][1].w};
-                uint32_t lo, hi, sb;
-                quantize_block16<true>(w8, s_enc, ftab, lo, hi, sb);
-                *reinterpret_cast<uint2 *>(xs + 8u * i) = make_uint2(lo, hi);
-                xs_sf[i] = static_cast<uint8_t>(sb);
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t i = i0 + k * kPrologueThreads;
+                    v[k][0] = v[k][1] = make_uint4(0, 0, 0, 0);
+                    valid[k] = false;
+                    if (i < nblk) {
+                        const uint32_t m = i / per_row, rem = i - m * per_row;
+                        int ks = ks0 + static_cast<int>(rem >> 4);
+                        if (ks >= p.kst) ks -= p.kst;
+                        const uint32_t b = static_cast<uint32_t>(ks) * 16u + (rem & 15u);
+                        if (b < kb16) {   // a partial last K stage has fewer blocks
+                            const uint32_t gi = m * kb16 + b;   // block of X, row-major
+                            v[k][0] = __ldg(p.x + 2u * gi);
+                            v[k][1] = __ldg(p.x + 2u * gi + 1u);
+                            valid[k] = true;
+                        }
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    if (valid[k]) quant_entry(i0 + k * kPrologueThreads, v[k][0], v[k][1]);
             }
         }
         named_bar_sync(kBarTok, kPrologueThreads);   // tokens quantized
@@ -443,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // the swizzled image the MMA reads (16-byte chunks of a 128-byte
             // row XORed with the row index mod 8), scales into the 512-byte tiles
             const int qt = threadIdx.x - kQuant0 * 32;   // 0 .. 63
-            const uint32_t rowb = static_cast<uint32_t>(p.K / 2);
+            const uint32_t rowc = per_row * 8u;   // code bytes per token row in the buffer
             int stage = 0;
             uint32_t phase = 0;
             for (int64_t u = u0; u < u1; ++u) {
@@ -451,19 +496,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int ks = static_cast<int>(u - static_cast<int64_t>(tile) * p.kst);
                 if (!warp_mbar_wait(empty0 + 8u * stage, phase ^ 1u, abort_flag, p.err)) break;
                 const int natoms = min(4, p.sf_ktiles - 4 * ks);
+                const int so = ks >= ks0 ? ks - ks0 : ks - ks0 + p.kst;   // slot in the buffer
                 uint8_t *sB = smem + stage * kStageBytes + kABytes;
                 uint8_t *sSB = sB + kBBytes + kSfBytes;
                 const int chunks = natoms * 2;   // 16-byte code chunks per token row
                 for (int it = qt; it < p.M * chunks; it += kQuantThreads) {
                     const int m = it / chunks, c = it - m * chunks;
-                    const uint4 v = *reinterpret_cast<const uint4 *>(xs + m * rowb + ks * 128 + c * 16);
+                    const uint4 v = *reinterpret_cast<const uint4 *>(xs + m * rowc + so * 128 + c * 16);
                     *reinterpret_cast<uint4 *>(sB + m * 128 + ((c ^ (m & 7)) * 16)) = v;
                 }
                 for (int it = qt; it < p.M * natoms; it += kQuantThreads) {
                     const int m = it / natoms, t4 = it - m * natoms;
                     // scales of blocks 4 t4 .. 4 t4 + 3 of the stage, row m < 32
                     *reinterpret_cast<uint32_t *>(sSB + t4 * 512 + m * 16) =
-                        *reinterpret_cast<const uint32_t *>(xs_sf + m * kb16 + ks * 16 + t4 * 4);
+                        *reinterpret_cast<const uint32_t *>(xs_sf + m * per_row + so * 16 + t4 * 4);
                 }
                 fence_proxy_async_smem();   // the writes above are read by the tensor core
                 __syncwarp();
@@ -569,6 +615,16 @@ TcSplit tc_split(int64_t N, int64_t K, int num_sms) {
 
 }  // namespace
 
+size_t decode_tc_token_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
+    // a CTA's range holds floor(total / ctas) units or one more, so it meets
+    // at most that many K stages (or all kst of them); 144 bytes per token
+    // and K stage (128 of codes, 16 of scales)
+    const TcSplit d = tc_split(N, K, num_sms);
+    int64_t n_st = d.total / d.ctas + 1;
+    if (n_st > d.kst) n_st = d.kst;
+    return static_cast<size_t>((M * n_st * 144 + 15) / 16 * 16);
+}
+
 size_t decode_tc_partial_floats(int64_t N, int64_t K, int num_sms) {
     const TcSplit d = tc_split(N, K, num_sms);
     return static_cast<size_t>(d.tiles) * d.slots * kTokens * 128;
@@ -578,7 +634,7 @@ cudaError_t launch_decode_nvf4_tc(const CUtensorMap &tmap_w, const uint8_t *w_sf
                                   const float *s_enc_w, int64_t N, int64_t K, const void *x_bf16,
                                   int64_t M, void *y, void *scratch, unsigned *err, int num_sms,
                                   cudaStream_t s) {
-    const size_t tok = (static_cast<size_t>(M) * static_cast<size_t>(K) * 9u / 16u + 15u) / 16u * 16u;
+    const size_t tok = decode_tc_token_bytes(M, N, K, num_sms);
     if (M < 1 || M > kDecodeTcTokens || tok > kDecodeTcTokenSmem) return cudaErrorInvalidValue;
     const TcSplit d = tc_split(N, K, num_sms);
     TcParams p;

@@ -158,8 +158,9 @@ cudaError_t launch_decode_nvf4_gemv(const uint8_t *w_codes, const uint8_t *w_sf,
                                     int num_sms, cudaStream_t s);
 
 // W4A4 decode on the tcgen05 tensor cores (mq_decode_tc.cu) for up to
-// kDecodeTcTokens BF16 tokens x [M, K] whose NVFP4 form (M K 9 / 16 bytes)
-// fits in kDecodeTcTokenSmem; the kernel quantizes them itself.  tmap_w is
+// kDecodeTcTokens BF16 tokens x [M, K]; each CTA quantizes them itself over
+// the K stages it covers, which must fit in kDecodeTcTokenSmem
+// (decode_tc_token_bytes: bytes per CTA for M tokens on an [N, K] weight).  tmap_w is
 // the weight codes' tensor map (encode_codes_tmap).  The weight is read
 // before the wait on the preceding kernel: no kernel may write it just before
 // (packing ends with a memory set).  decode_tc_partial_floats is the FP32
@@ -167,6 +168,7 @@ cudaError_t launch_decode_nvf4_gemv(const uint8_t *w_codes, const uint8_t *w_sf,
 constexpr int64_t kDecodeTcTokens = 16;
 constexpr size_t kDecodeTcTokenSmem = 40 * 1024;
 size_t decode_tc_partial_floats(int64_t N, int64_t K, int num_sms);
+size_t decode_tc_token_bytes(int64_t M, int64_t N, int64_t K, int num_sms);
 cudaError_t launch_decode_nvf4_tc(const CUtensorMap &tmap_w, const uint8_t *w_sf,
                                   const float *s_enc_w, int64_t N, int64_t K, const void *x_bf16,
                                   int64_t M, void *y, void *scratch, unsigned *err, int num_sms,

@@ -37,10 +37,13 @@ def gpu_decode_nvfp4(x_cpu, W):
 # (the two shapes past 2^25 elements below, and 1 x 9000 x 4032 with a partial
 # last K stage); 5-8 tokens the FP16-MMA kernel, except on weights past 2^25
 # elements with M K <= 32768 (6 x 9000 x 4096, 8 x 8200 x 4096: tensor cores).
+# The tensor-core kernel quantizes in each CTA only the K stages its units
+# cover (a compact buffer: 13 x 1024 x 4096, 3 x 4100 x 8192, 1 x 9000 x 4032
+# with a partial last stage), which lets 16 tokens with K = 14336 fit it.
 SHAPES = [(1, 256, 256), (8, 300, 320), (3, 17, 64), (13, 1024, 4096), (1, 1, 128),
           (2, 64, 8192), (1, 16, 16384), (8, 4096, 14336), (5, 100, 448), (16, 520, 1024),
           (17, 200, 512), (1, 6144, 4096), (4, 1000, 2048), (1, 9000, 4096), (3, 4100, 8192),
-          (1, 9000, 4032), (12, 300, 960), (6, 9000, 4096), (8, 8200, 4096)]
+          (1, 9000, 4032), (12, 300, 960), (6, 9000, 4096), (8, 8200, 4096), (16, 2048, 14336)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES)
