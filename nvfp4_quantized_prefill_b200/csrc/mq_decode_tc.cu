@@ -390,17 +390,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (i < kBBytes || i >= kBBytes + kSfBytes)   // skip the weight scale slot
                     *reinterpret_cast<uint4 *>(sB + i) = make_uint4(0, 0, 0, 0);
         }
+        // max |X| over all tokens: every CTA reads all of X (from L2), 16
+        // loads in flight per thread (with 4, 8 tokens x K = 14336 took ~19
+        // dependent rounds of L2 latency)
         const uint32_t vecs = static_cast<uint32_t>(p.M) * static_cast<uint32_t>(p.K / 8);
         uint32_t mx = 0;
-        for (uint32_t i0 = j; i0 < vecs; i0 += 4u * kPrologueThreads) {
-            uint4 v[4];
+        for (uint32_t i0 = j; i0 < vecs; i0 += 16u * kPrologueThreads) {
+            uint4 v[16];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
+            for (int k = 0; k < 16; ++k) {
                 const uint32_t i = i0 + k * kPrologueThreads;
                 v[k] = i < vecs ? __ldg(p.x + i) : make_uint4(0, 0, 0, 0);
             }
 #pragma unroll
-            for (int k = 0; k < 4; ++k) mx = max(mx, absmax8_bits(v[k]));
+            for (int k = 0; k < 16; ++k) mx = max(mx, absmax8_bits(v[k]));
         }
         mx = __reduce_max_sync(0xFFFFFFFFu, mx);
         if (lane == 0) red[j >> 5] = __uint_as_float(mx << 16);
