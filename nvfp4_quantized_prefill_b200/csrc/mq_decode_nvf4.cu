@@ -218,8 +218,17 @@ __global__ void __launch_bounds__(kPWarps * 32, 1) decode_nvf4_persist_kernel(
         const uint32_t vecs = static_cast<uint32_t>(M) * static_cast<uint32_t>(K / 8);
         const uint4 *xv = reinterpret_cast<const uint4 *>(xb);
         uint32_t mx = 0;
-#pragma unroll 4
-        for (uint32_t i = threadIdx.x; i < vecs; i += kPWarps * 32) mx = max(mx, absmax8_bits(__ldg(xv + i)));
+        // 8 loads in flight per thread (X comes from L2 in every CTA)
+        for (uint32_t i0 = threadIdx.x; i0 < vecs; i0 += 8u * kPWarps * 32) {
+            uint4 v[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t i = i0 + k * kPWarps * 32;
+                v[k] = i < vecs ? __ldg(xv + i) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) mx = max(mx, absmax8_bits(v[k]));
+        }
         mx = __reduce_max_sync(0xFFFFFFFFu, mx);
         if (lane == 0) red[warp] = __uint_as_float(mx << 16);
         __syncthreads();
@@ -232,14 +241,30 @@ __global__ void __launch_bounds__(kPWarps * 32, 1) decode_nvf4_persist_kernel(
         __syncthreads();
         const uint32_t nblk = static_cast<uint32_t>(M) * kblk;
         uint8_t *scl = xsm + static_cast<uint32_t>(M) * rowb;
-        for (uint32_t i = threadIdx.x; i < nblk; i += kPWarps * 32) {
-            const uint4 *src = xv + static_cast<uint64_t>(i) * 2u;  // block i = 16 elements
-            const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
-            const uint32_t w8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-            uint32_t lo, hi, sb;
-            quantize_block16<true>(w8, s, ftab, lo, hi, sb);
-            *reinterpret_cast<uint2 *>(xsm + i * 8u) = make_uint2(lo, hi);
-            scl[i] = static_cast<uint8_t>(sb);
+        // four blocks' loads issued before their quantization
+        for (uint32_t i0 = threadIdx.x; i0 < nblk; i0 += 4u * kPWarps * 32) {
+            uint4 v[4][2];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t i = i0 + k * kPWarps * 32;
+                v[k][0] = v[k][1] = make_uint4(0, 0, 0, 0);
+                if (i < nblk) {
+                    const uint4 *src = xv + static_cast<uint64_t>(i) * 2u;  // block i = 16 elements
+                    v[k][0] = __ldg(src);
+                    v[k][1] = __ldg(src + 1);
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t i = i0 + k * kPWarps * 32;
+                if (i >= nblk) break;
+                const uint32_t w8[8] = {v[k][0].x, v[k][0].y, v[k][0].z, v[k][0].w,
+                                        v[k][1].x, v[k][1].y, v[k][1].z, v[k][1].w};
+                uint32_t lo, hi, sb;
+                quantize_block16<true>(w8, s, ftab, lo, hi, sb);
+                *reinterpret_cast<uint2 *>(xsm + i * 8u) = make_uint2(lo, hi);
+                scl[i] = static_cast<uint8_t>(sb);
+            }
         }
         __syncthreads();
     }
