@@ -682,13 +682,12 @@ mq_status mq_decode_linear_nvfp4(const mq_weight *w, const void *x_bf16, int64_t
                          mq::decode_tc_token_bytes(M, w->N, w->K, d->num_sms) <= mq::kDecodeTcTokenSmem;
     const size_t tok_bytes = static_cast<size_t>(M) * static_cast<size_t>(w->K) * 9u / 16u;
     // the tensor-core kernel (quantizes the tokens itself, one pass over the
-    // weight) for up to 4 tokens and for 9 to 16; for 5 to 8 only on weights
-    // past 2^25 elements with M K <= 32768: there its stream beats the FP16
-    // dequantization of the FP16-MMA kernel (8B gate/up, 5 tokens: 26.0
-    // against 31.0 us), while with a longer K every CTA quantizing all the
-    // tokens costs it more (8B down, 5 tokens: 26.0 against 21.0 us)
-    const bool tc_mid = w->N * w->K > (int64_t(1) << 25) && M * w->K <= 32768;
-    if (tc_fits && (M <= 4 || M > 8 || tc_mid))
+    // weight) for up to 4 tokens and for 9 to 16; 5 to 8 tokens go to the
+    // FP16-MMA kernel.  (On the 8B gate/up weight alone the tensor-core kernel
+    // is faster at 5-8 tokens, 26.4 against 31.0 us at 5, but followed by the
+    // down projection on the FP16-MMA kernel the pass took 62.7 us at 8
+    // tokens against 54.0 us with both on the FP16-MMA kernel.)
+    if (tc_fits && (M <= 4 || M > 8))
         return cuda_status(mq::launch_decode_nvf4_tc(w->tmap, w->sf, w->s_enc, w->N, w->K, x_bf16,
                                                      M, y_bf16, w->decode_scratch, d->err,
                                                      d->num_sms, stream));

@@ -22,9 +22,8 @@
 // per CTA (one CTA per SM), so every SM streams the same bytes.  Each CTA's
 // few stages are short next to its fixed path (set-up, the first TMA round
 // trip, the token quantization, the accumulator hand-off and the cross-CTA
-// reduction), so the library uses it for up to 4 tokens, for 9 to 16, and
-// for 5 to 8 on weights past 2^25 elements; for 5 to 8 tokens on smaller
-// weights the FP16-MMA kernel is faster.
+// reduction), so the library uses it for up to 4 tokens and for 9 to 16; for
+// 5 to 8 the FP16-MMA kernel is used.
 //
 // CTA roles (9 warps):
 //   warp 0     TMA producer: weight codes [128 x 128 B] (128-byte swizzle)

@@ -35,8 +35,8 @@ def gpu_decode_nvfp4(x_cpu, W):
 # stream (partial last 1024-K step: K = 256, 64, 128, 2048 ...); larger weights
 # with 1-4 tokens and 9-16 tokens (M K 9/16 <= 40 KB) the tensor-core kernel
 # (the two shapes past 2^25 elements below, and 1 x 9000 x 4032 with a partial
-# last K stage); 5-8 tokens the FP16-MMA kernel, except on weights past 2^25
-# elements with M K <= 32768 (6 x 9000 x 4096, 8 x 8200 x 4096: tensor cores).
+# last K stage); 5-8 tokens the FP16-MMA kernel (also on weights past 2^25
+# elements: 6 x 9000 x 4096, 8 x 8200 x 4096).
 # The tensor-core kernel quantizes in each CTA only the K stages its units
 # cover (a compact buffer: 13 x 1024 x 4096, 3 x 4100 x 8192, 1 x 9000 x 4032
 # with a partial last stage), which lets 16 tokens with K = 14336 fit it.
